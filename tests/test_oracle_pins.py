@@ -1,0 +1,436 @@
+"""Pins of the fp64 oracle against what the pages and mathematics fix.
+
+None of these tests re-types an oracle formula: each checks a closed form,
+a special case that reduces to a textbook or library routine, an invariant
+the pages state, a hand-worked fixture (tests/golden/) or a brute-force
+enumeration on a tiny input. A plausible slip in the oracle (a dropped term,
+a wrong sign or index, a transposed operand, a tie broken the wrong way)
+fails at least one of them; tests at the end plant such slips and check
+that they are caught.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import expit, ndtr
+
+import oracle
+from oracle import moe_oracle as om
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rank_mask(keys, K):
+    """Brute force: member iff fewer than K ids beat it (greater key, or an
+    equal key with a lower id). Independent of any sort."""
+    keys = np.asarray(keys, dtype=np.float64)
+    n = keys.shape[0]
+    out = np.zeros(n, dtype=bool)
+    for i in range(n):
+        beats = sum(1 for j in range(n)
+                    if keys[j] > keys[i] or (keys[j] == keys[i] and j < i))
+        out[i] = beats < K
+    return out
+
+
+# ----------------------------------------------------------------- router
+def test_router_one_hot_rows_pick_weight_columns():
+    # x = e_j gives z[s, i] = W_r[i, j] (a transposed W_r would not).
+    rng = np.random.default_rng(0)
+    E, d = 5, 7
+    W = rng.normal(size=(E, d))
+    x = np.eye(d)
+    z = om.router_logits(x, W)
+    assert z.shape == (d, E)
+    np.testing.assert_array_equal(z, W.T)
+
+
+def test_router_bias_and_gate_residual_terms():
+    # x = 0 isolates the two additive terms: z = b + lambda * z_prev.
+    rng = np.random.default_rng(1)
+    T, d, E = 4, 3, 6
+    b = rng.normal(size=E)
+    zp = rng.normal(size=(T, E))
+    z = om.router_logits(np.zeros((T, d)), np.ones((E, d)), b, zp, 0.5)
+    np.testing.assert_allclose(z, b[None, :] + 0.5 * zp, rtol=0, atol=1e-15)
+    z0 = om.router_logits(np.zeros((T, d)), np.ones((E, d)), None, zp, 0.0)
+    np.testing.assert_array_equal(z0, np.zeros((T, E)))
+
+
+def test_softmax_closed_forms():
+    # exp(ln n) = n, so z = ln(1..E) gives A = (1..E) / sum(1..E).
+    z = np.log(np.array([[1.0, 2.0, 3.0]]))
+    np.testing.assert_allclose(om.softmax_rows(z), [[1 / 6, 2 / 6, 3 / 6]], rtol=1e-15)
+    # Two experts: A_0 = logistic(z_0 - z_1).
+    rng = np.random.default_rng(2)
+    z2 = rng.normal(size=(50, 2)) * 4
+    np.testing.assert_allclose(om.softmax_rows(z2)[:, 0], expit(z2[:, 0] - z2[:, 1]),
+                               rtol=1e-13)
+    # Equal logits give the uniform distribution.
+    np.testing.assert_allclose(om.softmax_rows(np.full((3, 8), 7.5)), 1 / 8, rtol=1e-15)
+
+
+def test_softmax_rows_sum_to_one_and_positive():
+    rng = np.random.default_rng(3)
+    z = rng.normal(size=(200, 19)) * 10
+    A = om.softmax_rows(z)
+    assert np.all(A > 0)
+    np.testing.assert_allclose(A.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    # Adding a per-row constant leaves A unchanged; large offsets must not overflow.
+    np.testing.assert_allclose(om.softmax_rows(z + 800.0), A, rtol=1e-12)
+
+
+# ------------------------------------------------------------ token choice
+def test_topk_golden_ties():
+    for case in _golden("topk_ties.json")["cases"]:
+        z = np.array([case["z"]])
+        assert om.topk_token_choice(z, case["k"])[0].tolist() == case["idx"], case["why"]
+
+
+def test_topk_matches_brute_force_with_ties():
+    rng = np.random.default_rng(4)
+    for _ in range(200):
+        E = int(rng.integers(1, 9))
+        k = int(rng.integers(1, E + 1))
+        z = rng.integers(-2, 3, size=(1, E)).astype(np.float64)  # many ties
+        got = om.topk_token_choice(z, k)[0]
+        assert np.array_equal(np.sort(got), np.nonzero(_rank_mask(z[0], k))[0])
+        # Rank order: keys non-increasing, equal keys in ascending id.
+        for a, b in zip(got[:-1], got[1:]):
+            assert z[0, a] > z[0, b] or (z[0, a] == z[0, b] and a < b)
+
+
+def test_topk_every_subset_is_dominated():
+    # Exhaustive: the chosen set is the unique k-subset that no swap improves.
+    rng = np.random.default_rng(5)
+    E, k = 6, 3
+    z = rng.integers(0, 3, size=E).astype(np.float64)
+    chosen = set(om.topk_token_choice(z[None], k)[0].tolist())
+
+    def better(i, j):
+        return z[i] > z[j] or (z[i] == z[j] and i < j)
+
+    winners = [set(S) for S in itertools.combinations(range(E), k)
+               if all(better(i, j) for i in S for j in range(E) if j not in S)]
+    assert winners == [chosen]
+
+
+def test_gather_weights_and_renorm():
+    A = np.array([[0.1, 0.6, 0.3]])
+    idx = np.array([[1, 2]])
+    np.testing.assert_array_equal(om.gather_weights(A, idx), [[0.6, 0.3]])
+    np.testing.assert_allclose(om.renormalize(np.array([[0.6, 0.3]])), [[2 / 3, 1 / 3]])
+
+
+# ----------------------------------------------------------- expert choice
+def test_capacity_closed_forms():
+    assert om.capacity(128, 32, 2.0) == 8       # the EC-DiT workload
+    assert om.capacity(8192, 32, 2.0) == 512    # whole-batch routing group
+    assert om.capacity(10, 4, 1.0) == 2         # 2.5 floors to 2
+    assert om.capacity(4, 8, 1.0) == 1          # 0.5 clamps up to 1
+    assert om.capacity(16, 4, 4.0) == 16        # f_c = E gives C = S
+
+
+def test_expert_choice_golden():
+    g = _golden("expert_choice_small.json")
+    assert om.capacity(g["group_size"], len(g["A"][0]), g["f_c"]) == g["C"]
+    tok, w = om.expert_choice(np.array(g["A"]), g["group_size"], g["C"])
+    assert tok.tolist() == g["tok"], g["why"]
+    np.testing.assert_array_equal(w, g["w"])
+
+
+def test_expert_choice_exactly_C_and_brute_force():
+    rng = np.random.default_rng(6)
+    G, S, E = 3, 12, 4
+    C = om.capacity(S, E, 2.0)
+    A = om.softmax_rows(rng.integers(0, 3, size=(G * S, E)).astype(float))  # ties
+    tok, w = om.expert_choice(A, S, C)
+    assert tok.shape == (G, E, C)
+    for g in range(G):
+        for e in range(E):
+            col = A[g * S:(g + 1) * S, e]
+            expect = g * S + np.nonzero(_rank_mask(col, C))[0]
+            assert np.array_equal(tok[g, e], expect)          # ascending, exact set
+            np.testing.assert_array_equal(w[g, e], A[tok[g, e], e])
+
+
+def test_expert_choice_full_capacity_takes_every_token():
+    # f_c = E gives C = S: every expert processes every token of its group.
+    rng = np.random.default_rng(7)
+    S, E = 8, 4
+    C = om.capacity(S, E, float(E))
+    A = om.softmax_rows(rng.normal(size=(2 * S, E)))
+    tok, _ = om.expert_choice(A, S, C)
+    for g in range(2):
+        for e in range(E):
+            assert tok[g, e].tolist() == list(range(g * S, (g + 1) * S))
+
+
+# ---------------------------------------------------------------- DES-Vote
+@pytest.mark.parametrize("name", ["des_vote_small.json", "des_vote_ties.json"])
+def test_des_vote_golden(name):
+    g = _golden(name)
+    votes, core, idx, w = om.des_vote(np.array(g["P"]), g["K"], g["M_core"])
+    q = [int(np.rint(v * 2.0 ** 40)) for v in g["votes_real"]]
+    # The fixture's real-valued totals, in the fixed point, up to one quantum per vote.
+    assert np.all(np.abs(votes - np.array(q)) <= len(g["P"])), g["why"]
+    assert core.tolist() == g["core"], g["why"]
+    assert idx.tolist() == g["idx"], g["why"]
+    np.testing.assert_array_equal(w.reshape(-1), g["w"])
+
+
+def test_vote_quantum_is_exact_fixed_point():
+    assert om.vote_quantum(0.5) == 2 ** 39
+    assert om.vote_quantum(1.0) == 2 ** 40
+    assert om.vote_quantum(2.0 ** -41) == 0          # half a quantum: ties to even (0)
+    assert om.vote_quantum(3 * 2.0 ** -41) == 2      # 1.5 quanta -> 2
+    p = np.float32(0.123456789)
+    assert om.vote_quantum(p) == int(np.float64(p) * 2 ** 40)  # exact: p has 24 bits
+
+
+def test_des_vote_brute_force_tally():
+    rng = np.random.default_rng(8)
+    N, M, K, Mc = 6, 10, 3, 5
+    P = om.softmax_rows(rng.integers(0, 4, size=(N, M)).astype(float))
+    votes, core, idx, w = om.des_vote(P, K, Mc)
+    V = [0] * M
+    for n in range(N):
+        mask = _rank_mask(P[n], K)
+        for e in range(M):
+            if mask[e]:
+                V[e] += int(np.rint(P[n, e] * 2.0 ** 40))
+    assert votes.tolist() == V
+    assert np.array_equal(core, np.nonzero(_rank_mask(np.array(V, dtype=float), Mc))[0])
+    for n in range(N):
+        sub = _rank_mask(P[n, core], K)
+        assert np.array_equal(np.sort(idx[n]), core[sub])
+
+
+def test_des_vote_beta_one_is_vanilla_topk():
+    # M_core = M: the core set is every expert, so re-routing is plain top-K.
+    rng = np.random.default_rng(9)
+    P = om.softmax_rows(rng.normal(size=(16, 12)))
+    votes, core, idx, w = om.des_vote(P, 4, om.des_core_size(12, 1.0))
+    assert core.tolist() == list(range(12))
+    assert np.array_equal(idx, om.topk_token_choice(P, 4))
+
+
+def test_des_vote_K_equals_M_gives_column_sums():
+    rng = np.random.default_rng(10)
+    P = om.softmax_rows(rng.normal(size=(7, 5)))
+    votes, _, _, _ = om.des_vote(P, 5, 5)
+    colsum = [sum(int(np.rint(P[n, e] * 2.0 ** 40)) for n in range(7)) for e in range(5)]
+    assert votes.tolist() == colsum
+
+
+def test_des_core_size_constant_over_block_size():
+    # DES page section 4.2: the number of active experts stays flat as the block grows.
+    rng = np.random.default_rng(11)
+    M, K = 64, 8
+    Mc = om.des_core_size(M, 0.5)
+    assert Mc == 32
+    for N in (1, 8, 16, 32, 64):
+        P = om.softmax_rows(rng.normal(size=(N, M)) + rng.normal(size=M)[None])
+        _, core, idx, _ = om.des_vote(P, K, Mc)
+        assert len(core) == Mc and len(set(core.tolist())) == Mc
+        assert set(np.unique(idx).tolist()) <= set(core.tolist())
+
+
+# ---------------------------------------------------------------- dispatch
+def test_dispatch_hand_example():
+    # Token choice, T=3, k=2, experts 0..2 heavy, 3 is zero-compute.
+    idx = np.array([[2, 0], [0, 3], [2, 1]])
+    a_tok = np.repeat(np.arange(3), 2)
+    offsets, perm, row_of, tok_ptr, tok_assign = om.dispatch(a_tok, idx.reshape(-1), 3, 3)
+    assert offsets.tolist() == [0, 2, 3, 5]          # e0: tokens 0,1; e1: 2; e2: 0,2
+    assert perm.tolist() == [0, 1, 2, 0, 2]
+    assert row_of.tolist() == [3, 0, 1, -1, 4, 2]
+    assert tok_ptr.tolist() == [0, 2, 4, 6]
+    assert tok_assign.tolist() == [0, 1, 2, 3, 4, 5]
+
+
+def test_dispatch_is_stable_bijection():
+    rng = np.random.default_rng(12)
+    T, k, E, Eh = 50, 3, 9, 6
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    a_tok = np.repeat(np.arange(T), k)
+    a_exp = idx.reshape(-1)
+    offsets, perm, row_of, tok_ptr, tok_assign = om.dispatch(a_tok, a_exp, Eh, T)
+    heavy = np.nonzero(a_exp < Eh)[0]
+    assert sorted(row_of[heavy].tolist()) == list(range(len(heavy)))
+    assert np.all(row_of[a_exp >= Eh] == -1)
+    for e in range(Eh):
+        toks = perm[offsets[e]:offsets[e + 1]]
+        assert len(toks) == int(np.sum(a_exp == e))
+        assert np.all(np.diff(toks) > 0)
+    for a in heavy:
+        assert perm[row_of[a]] == a_tok[a]
+    for s in range(T):
+        assert tok_assign[tok_ptr[s]:tok_ptr[s + 1]].tolist() == list(range(s * k, s * k + k))
+
+
+# ----------------------------------------------------------------- experts
+def test_gelu_textbook_values():
+    # GELU(u) = u * Phi(u); Phi(1) = 0.8413447460685429 (standard normal table).
+    assert om.gelu_erf(0.0) == 0.0
+    assert abs(om.gelu_erf(1.0) - 0.8413447460685429) < 1e-15
+    assert abs(om.gelu_erf(-1.0) + 0.15865525393145707) < 1e-15
+    u = np.linspace(-8, 8, 101)
+    np.testing.assert_allclose(om.gelu_erf(u), u * ndtr(u), rtol=1e-13, atol=1e-300)
+
+
+def test_silu_textbook_values():
+    assert om.silu(0.0) == 0.0
+    assert abs(om.silu(1.0) - 0.7310585786300049) < 1e-15
+    u = np.linspace(-20, 20, 81)
+    np.testing.assert_allclose(om.silu(u), u * expit(u), rtol=1e-13)
+
+
+def test_mlp_rank_one_closed_form():
+    # h = 1: W1 = a^T, W2 = b, so y = b * GELU(a . x) for every row.
+    rng = np.random.default_rng(13)
+    d = 5
+    a, b = rng.normal(size=d), rng.normal(size=d)
+    X = rng.normal(size=(4, d))
+    y = om.mlp_gelu(X, a[None, :], b[:, None])
+    expect = np.stack([b * (X[i] @ a) * ndtr(X[i] @ a) for i in range(4)])
+    np.testing.assert_allclose(y, expect, rtol=1e-13)
+    # SwiGLU with h = 1: y = c * silu(g . x) * (u . x).
+    g, u, c = rng.normal(size=d), rng.normal(size=d), rng.normal(size=d)
+    y2 = om.mlp_swiglu(X, g[None], u[None], c[:, None])
+    expect2 = np.stack([c * (X[i] @ g) * expit(X[i] @ g) * (X[i] @ u) for i in range(4)])
+    np.testing.assert_allclose(y2, expect2, rtol=1e-13)
+
+
+def test_mlp_identity_weights_give_activation():
+    X = np.linspace(-3, 3, 12).reshape(3, 4)
+    np.testing.assert_allclose(om.mlp_gelu(X, np.eye(4), np.eye(4)), X * ndtr(X), rtol=1e-14)
+
+
+def test_zero_compute_experts_return_x_zero_v():
+    rng = np.random.default_rng(14)
+    X = rng.normal(size=(5, 6))
+    v = rng.normal(size=6)
+    np.testing.assert_array_equal(om.zero_compute_expert(om.IDENTITY, X), X)
+    np.testing.assert_array_equal(om.zero_compute_expert(om.ZERO, X), 0.0)
+    np.testing.assert_array_equal(om.zero_compute_expert(om.CONST, X, v), np.tile(v, (5, 1)))
+
+
+# ------------------------------------------------------------- whole layer
+def _tiny(routing, E=6, kinds=None, shared=False, act="gelu", seed=0):
+    rng = np.random.default_rng(seed)
+    T, d, h = 24, 8, 16
+    kinds = kinds or [om.HEAVY] * E
+    Eh = sum(1 for k in kinds if k == om.HEAVY)
+    cfg = dict(routing=routing, E=E, h=h, act=act, k=2, group_size=8,
+               capacity=om.capacity(8, E, 2.0), M_core=om.des_core_size(E, 0.5))
+    x = rng.normal(size=(T, d))
+    Wr = rng.normal(size=(E, d))
+    W1 = rng.normal(size=(Eh, 2 * h if act == "swiglu" else h, d)) * 0.3
+    W2 = rng.normal(size=(Eh, d, h)) * 0.3
+    cv = rng.normal(size=(sum(1 for k in kinds if k == om.CONST), d))
+    Ws1 = rng.normal(size=(2 * h, d)) * 0.3 if shared else None
+    Ws2 = rng.normal(size=(d, 2 * h)) * 0.3 if shared else None
+    return cfg, x, Wr, W1, W2, kinds, cv, Ws1, Ws2
+
+
+def _mask(cfg, sel, T):
+    a_tok, a_exp, _ = om.assignments_from_selection(cfg, sel)
+    m = np.zeros((T, cfg["E"]))
+    m[a_tok, a_exp] = 1
+    return m
+
+
+@pytest.mark.parametrize("routing,act,shared,kinds", [
+    ("token_topk", "gelu", False, None),
+    ("token_topk", "gelu", True, [0, 0, 0, 1, 2, 3]),
+    ("expert_choice", "gelu", False, None),
+    ("des_vote", "swiglu", False, None),
+])
+def test_forward_equals_dense_masked_sum(routing, act, shared, kinds):
+    cfg, x, Wr, W1, W2, kinds, cv, Ws1, Ws2 = _tiny(routing, kinds=kinds, shared=shared, act=act)
+    sel = om.route(cfg, x, Wr)
+    y = om.forward(cfg, x, W1, W2, sel, kinds, cv, Ws1, Ws2, residual=x)
+    yd = om.dense_masked_forward(cfg, x, W1, W2, sel["A"], _mask(cfg, sel, x.shape[0]),
+                                 kinds, cv, Ws1, Ws2, residual=x)
+    np.testing.assert_allclose(y, yd, rtol=1e-12, atol=1e-12)
+    # A subset of tokens gives exactly those rows.
+    sub = np.array([3, 0, 17])
+    ys = om.forward(cfg, x, W1, W2, sel, kinds, cv, Ws1, Ws2, residual=x, tokens=sub)
+    np.testing.assert_allclose(ys, y[sub], rtol=1e-13, atol=1e-13)
+
+
+def test_single_expert_layer_is_textbook_mlp():
+    # E = 1, k = 1: softmax over one expert is 1, so y = x + W2 GELU(W1 x).
+    rng = np.random.default_rng(15)
+    T, d, h = 10, 6, 12
+    x = rng.normal(size=(T, d))
+    W1, W2 = rng.normal(size=(1, h, d)), rng.normal(size=(1, d, h))
+    cfg = dict(routing="token_topk", E=1, h=h, act="gelu", k=1)
+    sel = om.route(cfg, x, rng.normal(size=(1, d)))
+    np.testing.assert_array_equal(sel["w"], 1.0)
+    y = om.forward(cfg, x, W1, W2, sel, residual=x)
+    hid = x @ W1[0].T
+    np.testing.assert_allclose(y, x + (hid * ndtr(hid)) @ W2[0].T, rtol=1e-12)
+
+
+def test_zero_compute_routes_through_layer():
+    # Route every token to one zero-compute expert with weight 1.
+    rng = np.random.default_rng(16)
+    T, d = 6, 4
+    x = rng.normal(size=(T, d))
+    v = rng.normal(size=(1, d))
+    kinds = [om.HEAVY, om.IDENTITY, om.ZERO, om.CONST]
+    cfg = dict(routing="token_topk", E=4, h=3, act="gelu", k=1)
+    W1, W2 = np.zeros((1, 3, d)), np.zeros((1, d, 3))
+    for e, expect in ((1, x + x), (2, x), (3, x + v)):
+        sel = {"idx": np.full((T, 1), e), "w": np.ones((T, 1))}
+        y = om.forward(cfg, x, W1, W2, sel, kinds, v, residual=x)
+        np.testing.assert_array_equal(y, expect)
+
+
+def test_shared_concatenation_equals_sum_of_experts():
+    # Two shared experts concatenated along the hidden dim are their sum.
+    rng = np.random.default_rng(17)
+    d, h = 5, 7
+    X = rng.normal(size=(3, d))
+    A1, A2 = rng.normal(size=(h, d)), rng.normal(size=(h, d))
+    B1, B2 = rng.normal(size=(d, h)), rng.normal(size=(d, h))
+    cat = om.mlp_gelu(X, np.vstack([A1, A2]), np.hstack([B1, B2]))
+    sep = om.mlp_gelu(X, A1, B1) + om.mlp_gelu(X, A2, B2)
+    np.testing.assert_allclose(cat, sep, rtol=1e-12)
+
+
+# ---------------------------------------------- planted slips are caught
+def test_planted_tie_flip_is_caught(monkeypatch):
+    # Plant "ties go to the higher id" in the oracle and check a pin fails.
+    monkeypatch.setattr(om, "_order_desc", lambda keys, ids: np.lexsort((-np.asarray(ids), -np.asarray(keys, float))))
+    case = _golden("topk_ties.json")["cases"][0]
+    assert om.topk_token_choice(np.array([case["z"]]), case["k"])[0].tolist() != case["idx"]
+
+
+def test_planted_softmax_axis_slip_is_caught(monkeypatch):
+    def bad(z):
+        z = np.asarray(z, float)
+        e = np.exp(z - z.max(axis=0, keepdims=True))
+        return e / e.sum(axis=0, keepdims=True)
+    monkeypatch.setattr(om, "softmax_rows", bad)
+    z = np.log(np.array([[1.0, 2.0, 3.0], [1.0, 1.0, 1.0]]))
+    assert not np.allclose(om.softmax_rows(z).sum(axis=1), 1.0)
+
+
+def test_planted_vote_without_filter_is_caught():
+    # Voting with all experts (no top-K filter) changes the small fixture.
+    g = _golden("des_vote_small.json")
+    P = np.array(g["P"])
+    unfiltered = (P * 2.0 ** 40).sum(axis=0)
+    assert int(np.argmax(unfiltered)) == 0 and unfiltered[3] != g["votes_real"][3] * 2 ** 40
