@@ -1,0 +1,454 @@
+"""Benchmark of the MoE-layer forward pass on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
+
+A step is one pass of the whole layer (router + softmax + selection ->
+dispatch -> grouped expert MLP -> combine) over one batch of synthetic input,
+issued as the library's staged C-ABI calls on one stream with a CUDA event
+between stages; the same launches moe_forward makes. L2 is flushed (a
+256 MiB write) before every timed step, outside the events. ``value`` is
+tokens/s over the K timed steps (inputs resident in HBM); ``e2e`` repeats
+the measurement through moe_forward_host with the activations in pinned
+host memory and the copies inside the timed region. Multi-GPU runs are
+independent replicas (one process per GPU, no collective on the data path);
+the time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "ditmoe_xl"
+METRIC = "MoE-layer tokens/s and TFLOP/s (or HBM GB/s) vs B200 roofline, 1 GPU"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------- bookkeeping
+def describe(cfg):
+    """Workload description for the JSON line."""
+    parts = [f"T={cfg['T']}", f"d={cfg['d']}", f"E={cfg['E']}"]
+    if cfg["routing"] == "token_topk":
+        parts.append(f"top-{cfg['k']}")
+    elif cfg["routing"] == "expert_choice":
+        parts.append(f"expert-choice S={cfg['group_size']} C={cfg['capacity']}")
+    else:
+        parts.append(f"DES-Vote K={cfg['k']} M_core={cfg['M_core']}")
+    parts.append(f"h={cfg['h']} {cfg['act']}")
+    if cfg["n_shared"]:
+        parts.append(f"+{cfg['n_shared']} shared h={cfg['h_shared']}")
+    if cfg["E_heavy"] != cfg["E"]:
+        parts.append(f"{cfg['E'] - cfg['E_heavy']} zero-compute experts")
+    return f"{cfg['name']}: " + ", ".join(parts) + f", {cfg['dtype']}"
+
+
+def mlp_flops(cfg, n_heavy_rows):
+    """Algorithmic FLOPs of the grouped MLP: executed heavy rows and shared tokens only."""
+    gemm = 6 if cfg["act"] == "swiglu" else 4  # 2*d*h per GEMM; SwiGLU has gate+up+down
+    routed = n_heavy_rows * gemm * cfg["d"] * cfg["h"]
+    shared = cfg["T"] * 4 * cfg["d"] * cfg["n_shared"] * cfg["h_shared"]
+    return routed + shared
+
+
+def weight_bytes_used(cfg, used_experts):
+    """Unique heavy-expert weight bytes one layer pass must read (DES latency model)."""
+    per = (3 if cfg["act"] == "swiglu" else 2) * cfg["d"] * cfg["h"] * (2 if cfg["dtype"] == "bf16" else 4)
+    return used_experts * per
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def reduce_max_over_ranks(value, dist=None):
+    """Max of a float over all ranks (identity without a process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank, world, max_seconds):
+    return units_per_rank * world / max_seconds
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                cols = [c.strip() for c in line.split(",")]
+                if len(cols) < 9:
+                    continue
+                try:
+                    sm.append(float(cols[1]))
+                    smax = float(cols[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, cols[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------- GPU benchmark
+class StagedLayer:
+    """One layer pass as staged C-ABI calls with an event between stages."""
+
+    def __init__(self, m, cfg, inp, device):
+        import torch
+        self.m, self.cfg, self.inp = m, cfg, inp
+        self.c = m.make_config(cfg)
+        na = m.num_assignments(self.c)
+        T, E, d = cfg["T"], cfg["E"], cfg["d"]
+        f = dict(device=device)
+        self.logits = torch.empty(T, E, dtype=torch.float32, **f)
+        self.probs = torch.empty(T, E, dtype=torch.float32, **f)
+        self.sel = torch.empty(na, dtype=torch.int32, **f)
+        self.w = torch.empty(na, dtype=torch.float32, **f)
+        self.votes = torch.empty(E, dtype=torch.int64, **f)
+        self.core = torch.empty(max(1, cfg.get("M_core", 0)), dtype=torch.int32, **f)
+        self.offsets = torch.empty(self.c.n_heavy + 1, dtype=torch.int32, **f)
+        self.perm = torch.empty(na, dtype=torch.int32, **f)
+        self.row_of = torch.empty(na, dtype=torch.int32, **f)
+        ec = cfg["routing"] == "expert_choice"
+        self.tok_ptr = torch.empty(T + 1, dtype=torch.int32, **f) if ec else None
+        self.tok_assign = torch.empty(na, dtype=torch.int32, **f) if ec else None
+        self.x_perm = torch.empty(na, d, dtype=inp["x"].dtype, **f)
+        self.y_perm = torch.empty(na, d, dtype=torch.float32, **f)
+        self.y_sh = torch.empty(T, d, dtype=torch.float32, **f) if cfg["n_shared"] else None
+        self.y = torch.empty_like(inp["x"])
+        self.ws = m.alloc_workspace(self.c, device)
+        self.status = torch.zeros(1, dtype=torch.int32, **f)
+        self.stages = ["router+select", "dispatch", "grouped_mlp", "combine"]
+        self.launches = {"router+select": 1 + (cfg["routing"] != "token_topk"),
+                         "dispatch": 4 + (1 if ec else 0),
+                         "grouped_mlp": 2,
+                         "combine": 1}
+        if cfg["n_shared"] and (cfg["dtype"] != "bf16" or cfg["act"] != "gelu"):
+            self.launches["grouped_mlp"] = 3 if cfg["dtype"] == "bf16" else 4
+
+    def run(self, events=None):
+        m, cfg, i = self.m, self.cfg, self.inp
+        r = cfg["routing"]
+
+        def mark(j):
+            if events is not None:
+                events[j].record()
+        mark(0)
+        m.router(i["x"], i["W_r"], self.logits, self.probs, bias=i["logit_bias"],
+                 z_prev=i["z_prev"], z_prev_scale=cfg["gate_residual_scale"],
+                 k=cfg["k"] if r == "token_topk" else 0, renorm=cfg["renorm"],
+                 idx=self.sel if r == "token_topk" else None,
+                 w=self.w if r == "token_topk" else None)
+        if r == "expert_choice":
+            m.select_expert_choice(self.probs, cfg["group_size"], cfg["capacity"], self.sel, self.w)
+        elif r == "des_vote":
+            m.core_set_vote(self.probs, cfg["k"], cfg["M_core"], self.votes, self.core, self.sel, self.w)
+        mark(1)
+        m.dispatch(self.c, self.sel, i["x"], self.x_perm, self.offsets, self.perm, self.row_of,
+                   self.tok_ptr, self.tok_assign, self.status, self.ws)
+        mark(2)
+        m.grouped_mlp(self.c, self.x_perm, self.offsets, i["W1"], i["W2"], i["x"], i["Ws1"],
+                      i["Ws2"], self.y_perm, self.y_sh, self.status, self.ws)
+        mark(3)
+        m.combine(self.c, self.y_perm, self.y_sh, self.sel, self.w, self.row_of, self.tok_ptr,
+                  self.tok_assign, i["x"], i["const_vecs"], i["x"], self.y, self.status)
+        mark(4)
+
+
+def gpu_bench(args):
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_33_b200 import inputs as gen
+    from mixture_experts_layer_33_b200 import moe as m
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if m.device_check(local) != m.MOE_OK:
+        raise RuntimeError("not an sm_100 GPU")
+
+    cfg = gen.workload(args.workload)
+    inp = gen.make_inputs(cfg, dev)
+    layer = StagedLayer(m, cfg, inp, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        layer.run()
+    torch.cuda.synchronize()
+    if int(layer.status.item()) != 0:
+        raise RuntimeError(f"device status {int(layer.status.item())}")
+
+    # Executed heavy rows and used experts (fixed by the seeded inputs).
+    offs = layer.offsets.cpu().tolist()
+    n_rows = offs[-1]
+    used = sum(1 for a, b in zip(offs[:-1], offs[1:]) if b > a)
+    flops = mlp_flops(cfg, n_rows)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.fill_(s & 255)
+        layer.run(ev[s])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    stage_ms = {n: 0.0 for n in layer.stages}
+    total_ms = 0.0
+    for s in range(args.steps):
+        for j, n in enumerate(layer.stages):
+            t = ev[s][j].elapsed_time(ev[s][j + 1])
+            stage_ms[n] += t
+            total_ms += t
+    max_s = reduce_max_over_ranks(total_ms / 1e3, dist if world > 1 else None)
+    ms_per_step = max_s * 1e3 / args.steps
+    value = aggregate_throughput(cfg["T"] * args.steps, world, max_s)
+
+    # End to end through moe_forward_host: pinned host activations, copies timed.
+    x_h = inp["x"].cpu().pin_memory()
+    zp_h = inp["z_prev"].cpu().pin_memory() if inp["z_prev"] is not None else None
+    y_h = torch.empty_like(x_h).pin_memory()
+    ws = m.alloc_workspace(layer.c, dev)
+
+    def e2e_step():
+        m.forward_host(layer.c, x_h, inp["W_r"], inp["W1"], inp["W2"], y_h, ws,
+                       residual_host=x_h, z_prev_host=zp_h, bias=inp["logit_bias"],
+                       Ws1=inp["Ws1"], Ws2=inp["Ws2"], const_vecs=inp["const_vecs"],
+                       dev_status=layer.status)
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = 0.0
+    for s in range(args.steps):
+        flush.fill_(s & 255)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    e2e_s = reduce_max_over_ranks(e2e_ms / 1e3, dist if world > 1 else None)
+    act_bytes = cfg["T"] * cfg["d"] * inp["x"].element_size()
+    h2d = act_bytes + (cfg["T"] * cfg["E"] * 4 if zp_h is not None else 0)
+
+    peaks, peak_src = load_peaks()
+    gm_ms = stage_ms["grouped_mlp"] / args.steps
+    if cfg["routing"] == "des_vote":
+        bytes_ = weight_bytes_used(cfg, used)
+        achieved = bytes_ / (gm_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": "grouped_mlp (GEMM1 + GEMM2 launches)",
+                "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "algorithmic_per_launch": bytes_, "peak_source": peak_src}
+    else:
+        achieved = flops / (gm_ms / 1e3) / 1e12
+        pk = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "kernel": "grouped_mlp (GEMM1 + GEMM2 launches)",
+                "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
+                "frac": round(achieved / pk, 4), "traffic": None,
+                "algorithmic_per_launch": flops, "peak_source": peak_src + " (burst)"}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": cfg["dtype"], "data": "synthetic (seeded Gaussian inputs, random-init weights)",
+        "config": {"workload": describe(cfg), "global_batch_tokens": cfg["T"] * world,
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "flushed by a 256 MiB write before every timed step"},
+        "layer_tflops": round(flops / (ms_per_step / 1e3) / 1e12, 1),
+        "stage_ms": {k: round(v / args.steps, 4) for k, v in stage_ms.items()},
+        "heavy_rows": n_rows, "experts_used": used,
+        "roofline": roof,
+        "e2e": {"value": round(aggregate_throughput(cfg["T"] * args.steps, world, e2e_s), 1),
+                "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": act_bytes,
+                "api": "moe_forward_host"},
+        "gpu_launches": sum(layer.launches.values()) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, {k: gen.to_numpy_f32(v) for k, v in inp.items()},
+                                            budget_s=args.cpu_budget)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------- oracle (CPU) timing
+def _oracle_sample(cfg, hin, n_tokens):
+    """The oracle's full layer (its own fp64 routing) on the first tokens.
+
+    Token choice: per-token routing, so any prefix is exact. Expert choice:
+    whole routing groups. DES: the whole block.
+    """
+    import oracle
+    if cfg["routing"] == "expert_choice":
+        S = cfg["group_size"]
+        n_tokens = max(S, (n_tokens // S) * S)
+    if cfg["routing"] == "des_vote":
+        n_tokens = cfg["T"]
+    n = min(n_tokens, cfg["T"])
+    sub = dict(cfg, T=n)
+    zp = hin["z_prev"][:n] if hin["z_prev"] is not None else None
+    sel = oracle.route(sub, hin["x"][:n], hin["W_r"], hin["logit_bias"], zp)
+    y = oracle.forward(sub, hin["x"][:n], hin["W1"], hin["W2"], sel, cfg["kinds"],
+                       hin["const_vecs"], hin["Ws1"], hin["Ws2"], residual=hin["x"][:n])
+    return n, y
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(cfg, hin, budget_s=15.0):
+    """Time the oracle as it stands on a bounded sample (grows until ~budget_s)."""
+    n = 64 if cfg["routing"] == "token_topk" else 1
+    best = None
+    t_total = 0.0
+    while True:
+        t0 = time.perf_counter()
+        done, _ = _oracle_sample(cfg, hin, n)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        best = (done, dt)
+        if done >= cfg["T"] or dt >= budget_s / 3 or t_total >= budget_s:
+            break
+        n *= 2
+    done, dt = best
+    return {"value": round(done / dt, 2), "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, own routing, first {done} of {cfg['T']} tokens "
+                      f"({dt:.1f} s)"}
+
+
+def reference_bench(args):
+    """--impl reference: the oracle on the host cores, same metric/config."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    from mixture_experts_layer_33_b200 import inputs as gen
+    cfg = gen.workload(args.workload)
+    hin = {k: gen.to_numpy_f32(v) for k, v in gen.make_inputs(cfg, "cpu").items()}
+    # Per-step sample sized so K + W steps finish in a few minutes.
+    n = 64 if cfg["routing"] == "token_topk" else 1
+    t0 = time.perf_counter()
+    done, _ = _oracle_sample(cfg, hin, n)
+    probe = time.perf_counter() - t0
+    per_step_budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    if cfg["routing"] == "token_topk" and probe < per_step_budget:
+        n = int(n * min(64, per_step_budget / max(probe, 1e-3)))
+    for _ in range(args.warmup):
+        _oracle_sample(cfg, hin, n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        done, _ = _oracle_sample(cfg, hin, n)
+    dt = time.perf_counter() - t0
+    v = done * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(v, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(cfg)},
+        "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "cores": _cores(),
+                         "kind": "oracle",
+                         "sample": f"first {done} of {cfg['T']} tokens per step"},
+        "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "torch_threads": torch.get_num_threads(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference_bench(args)
+    else:
+        gpu_bench(args)
+
+
+if __name__ == "__main__":
+    main()

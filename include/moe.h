@@ -1,0 +1,307 @@
+/*
+ * moe.h - C ABI of libmoe.so, a B200 (sm_100a) MoE-layer forward pass.
+ *
+ * The layer (shared by DiT-MoE, EC-DiT, MMOE and the DES dLLM block):
+ *   router GEMM + softmax      -> affinities A in R^{T x E}
+ *   selection                  -> token-choice top-k | expert-choice top-C |
+ *                                 DES-Vote core set + restricted top-K
+ *   dispatch                   -> stable permutation into per-expert groups
+ *   grouped expert MLP         -> GELU or SwiGLU heavy experts (tcgen05 tensor
+ *                                 cores for bf16), shared expert(s); the
+ *                                 zero-computation experts issue no FLOPs
+ *   combine                    -> y = r + shared + sum_j w_j * expert_j(x)
+ *
+ * Conventions for every entry point
+ *   - Returns an int moe_status (MOE_OK == 0); moe_status_string() names it.
+ *     Host-side argument checks run before anything is launched; a failing
+ *     check launches nothing.
+ *   - Tensor arguments are DEVICE pointers owned by the caller, row-major
+ *     and contiguous, unless a parameter says "host". bf16 rows must start
+ *     on 16-byte boundaries (row lengths d, h that are multiples of 8).
+ *   - Calls are asynchronous on the given stream (NULL = legacy default
+ *     stream) and never synchronise the host. Errors found on the device
+ *     (an expert or token index out of range, a bounded wait that expired)
+ *     are OR-ed into the caller's int32 status word `dev_status` (device
+ *     memory, nullable) as MOE_DEV_* bits; the offending item is skipped,
+ *     nothing traps.
+ *   - The library allocates no memory. Scratch comes from a caller
+ *     workspace of at least moe_workspace_size() bytes, 256-byte aligned.
+ *     Calls that share a workspace must not overlap on the device.
+ *   - There is no global mutable state: calls on different streams with
+ *     different workspaces may run concurrently.
+ *
+ * Expert ids: heavy (MLP) experts occupy ids [0, n_heavy); ids
+ * [n_heavy, E) are zero-computation experts whose kinds are listed in
+ * moe_config.expert_kind (MMOE page, "MoE++ expert layer").
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st *moe_stream_t; /* a cudaStream_t */
+
+enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, size out of range, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. E > 256, not sm_100) */
+  MOE_ERR_WORKSPACE = 3,     /* workspace smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_STATUS = 5, /* reserved for callers reporting a nonzero dev_status */
+  MOE_ERR_TIMEOUT = 6        /* reserved for callers reporting MOE_DEV_TIMEOUT */
+};
+
+/* Bits OR-ed into dev_status by kernels. */
+#define MOE_DEV_BAD_EXPERT 1u /* a selected expert id outside [0, E) */
+#define MOE_DEV_BAD_TOKEN 2u  /* a selected token id outside [0, T) */
+#define MOE_DEV_TIMEOUT 4u    /* a bounded wait inside a kernel expired */
+#define MOE_DEV_OVERFLOW 8u   /* more rows than the caller's buffers hold */
+
+enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 };
+enum moe_routing { MOE_TOKEN_TOPK = 0, MOE_EXPERT_CHOICE = 1, MOE_DES_VOTE = 2 };
+enum moe_act { MOE_GELU_ERF = 0, MOE_SWIGLU = 1 };
+enum moe_expert_kind { MOE_HEAVY = 0, MOE_IDENTITY = 1, MOE_ZERO = 2, MOE_CONST = 3 };
+
+#define MOE_MAX_EXPERTS 256
+
+/*
+ * Layer configuration (host memory, read during the call only).
+ *
+ * T           tokens in the launch (for DES-Vote: the block's N tokens)
+ * d           model width; h heavy-expert hidden width
+ * E           routed experts of every kind (heavy + zero-computation)
+ * n_heavy     heavy experts, ids [0, n_heavy)
+ * k           token choice: experts per token; DES-Vote: the per-token K
+ * n_shared, h_shared  shared experts and their hidden width; they are
+ *             passed concatenated along the hidden dimension (n_shared *
+ *             h_shared hidden units), which for GELU experts equals the sum
+ *             of the separate experts exactly
+ * dtype       moe_dtype of x, weights, residual, y (router/selection in fp32)
+ * act         moe_act of the heavy experts (shared experts are GELU)
+ * routing     moe_routing
+ * group_size  expert choice: tokens S per routing group (T % S == 0)
+ * capacity    expert choice: tokens C chosen per expert per group
+ *             (EC-DiT page, "capacity factor": C = f_c * S / E)
+ * M_core      DES-Vote core-set size (DES page, section 3.1: beta * M)
+ * gate_residual_scale  weight of the previous layer's logits z_prev
+ * renorm      0: weights are the full-softmax affinities A (the pages'
+ *             definition); 1: renormalised over each token's selection
+ * expert_kind kinds of ids [0, E): MOE_HEAVY for ids < n_heavy, a
+ *             zero-computation kind for the others
+ */
+typedef struct moe_config {
+  int32_t T, d, h, E, n_heavy, k;
+  int32_t n_shared, h_shared;
+  int32_t dtype, act, routing;
+  int32_t group_size, capacity, M_core;
+  float gate_residual_scale;
+  int32_t renorm;
+  int32_t expert_kind[MOE_MAX_EXPERTS];
+} moe_config;
+
+/* Human-readable name of a moe_status. Never NULL. */
+MOE_API const char *moe_status_string(int status);
+
+/* MOE_OK if `device` is an sm_100 GPU this library was built for, else
+ * MOE_ERR_UNSUPPORTED (or MOE_ERR_CUDA if the device cannot be queried). */
+MOE_API int moe_device_check(int device);
+
+/* Number of routing assignments of a configuration: T*k for token choice
+ * and DES-Vote, (T/S)*E*C for expert choice. */
+MOE_API int moe_num_assignments(const moe_config *cfg, int64_t *n_assign);
+
+/* Workspace bytes moe_forward / moe_forward_host need for `cfg`
+ * (moe_dispatch and moe_grouped_mlp need at most this much). */
+MOE_API int moe_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/*
+ * Router GEMM, softmax and (optionally) token-choice top-k, fused.
+ * EC-DiT page, section 3 "Expert-Choice routing formula": given x' in
+ * R^{S x d}, A_{s,i} = exp((x' W_r)_{s,i}) / sum_j exp((x' W_r)_{s,j}).
+ * MMOE page, "gate-residual routing": the previous expert layer's gate
+ * logits are carried into the router: z = x W_r + b + scale * z_prev.
+ *
+ *   x        [T, d] (dtype)         W_r [E, d] (dtype; row e = expert e)
+ *   bias     [E] fp32, nullable     z_prev [T, E] fp32, nullable
+ *   logits   [T, E] fp32 out (z)    probs [T, E] fp32 out (A)
+ *   k        0: no selection; else 1 <= k <= E and idx/w must be given
+ *   idx      [T, k] int32 out: top-k expert ids by z, descending, ties to
+ *            the lower id (EC-DiT page, "Token-Choice routing")
+ *   w        [T, k] fp32 out: A[s, idx] (renormalised if renorm)
+ * Limits: 1 <= E <= 128, d % 8 == 0 for bf16.
+ */
+MOE_API int moe_router(const void *x, const void *W_r, const float *bias,
+               const float *z_prev, float z_prev_scale, int T, int d, int E,
+               int dtype, float *logits, float *probs, int k, int renorm,
+               int32_t *idx, float *w, moe_stream_t stream);
+
+/*
+ * Token-choice top-k from given fp32 logits (the selection half of
+ * moe_router, for callers that hold their own logits).
+ * EC-DiT page, section 3 "Token-Choice routing": each token selects its
+ * top-k experts. Ranking key z, ties to the lower expert id; dropless.
+ *   logits [T, E], probs [T, E] fp32 in; idx [T, k] int32, w [T, k] fp32 out.
+ * Limits: 1 <= k <= E <= 128.
+ */
+MOE_API int moe_select_topk(const float *logits, const float *probs, int T, int E,
+                    int k, int renorm, int32_t *idx, float *w,
+                    moe_stream_t stream);
+
+/*
+ * Expert-choice top-C per expert column, by block radix select.
+ * EC-DiT page, section 3 "Expert-Choice routing" (each expert picks its
+ * top tokens) and "capacity factor" (Capacity = f_c * S / E). The routing
+ * group is one sequence of S = group_size tokens.
+ *   probs [T, E] fp32 in (A; T % S == 0)
+ *   tok   [T/S, E, C] int32 out: GLOBAL token ids in ascending order
+ *   w     [T/S, E, C] fp32 out: A[tok, e]
+ * Ranking key A, ties to the lower token id. Limits: 1 <= C <= S <= 16384.
+ */
+MOE_API int moe_select_expert_choice(const float *probs, int T, int E, int group_size,
+                             int C, int32_t *tok, float *w,
+                             moe_stream_t stream);
+
+/*
+ * DES-Vote core set and restricted re-routing, for one block of N tokens.
+ * Dynamic Expert Sharing page, section 2.4 "DES-Vote": each token masks to
+ * its own top-K experts, votes with their routing weights, and the M_core
+ * experts with the largest totals form the core set; section 4.3: tokens
+ * then re-activate K experts from the core set.
+ *   probs [N, M] fp32 in (P = A)
+ *   votes [M] int64 out: sum over tokens of q(P) for each token's top-K,
+ *         q(p) = round-half-even(p * 2^40) (exact, order-independent)
+ *   core  [M_core] int32 out: elected experts in ascending id order
+ *         (ranked by votes, ties to the lower id; always M_core entries)
+ *   idx   [N, K] int32 out: each token's K largest P over the core set,
+ *         descending, ties to the lower id;   w [N, K] fp32 out: P[n, idx]
+ * Limits: 1 <= K <= M_core <= M <= 256, N <= 4096.
+ */
+MOE_API int moe_core_set_vote(const float *probs, int N, int M, int K, int M_core,
+                      int64_t *votes, int32_t *core, int32_t *idx, float *w,
+                      moe_stream_t stream);
+
+/*
+ * Dispatch: a stable permutation of the heavy assignments into per-expert
+ * groups (histogram, exclusive scan, scatter), plus the gather of x rows.
+ * DICE page, "Conditional Communication" and the expert-parallel
+ * dispatch/combine it schedules: tokens go to their experts, outputs come
+ * back weighted by the routing score.
+ *
+ * Assignments in slot order a = 0..n_assign-1 come from `sel`:
+ *   token choice / DES: sel = idx [T, k]; a = s*k + j has token s, expert sel[a]
+ *   expert choice:      sel = tok [T/S, E, C]; a = (g*E + e)*C + c has
+ *                       token sel[a], expert e
+ * Outputs (device, caller-owned; sized for n_assign rows at most):
+ *   offsets    [n_heavy + 1] int32: rows of expert e are offsets[e]..offsets[e+1]
+ *   perm       [n_assign] int32: token of each row, ascending within an expert
+ *   row_of     [n_assign] int32: row of assignment a, -1 if not heavy
+ *   x_perm     [n_assign, d] (dtype), nullable: x_perm[r] = x[perm[r]]
+ *   tok_ptr    [T + 1], tok_assign [n_assign] int32, nullable, expert choice
+ *              only: each token's assignments in slot order (a CSR)
+ * Out-of-range ids set MOE_DEV_BAD_EXPERT / MOE_DEV_BAD_TOKEN and are dropped.
+ */
+MOE_API int moe_dispatch(const moe_config *cfg, const int32_t *sel, const void *x,
+                 void *x_perm, int32_t *offsets, int32_t *perm, int32_t *row_of,
+                 int32_t *tok_ptr, int32_t *tok_assign, int32_t *dev_status,
+                 void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Grouped expert MLP over the dispatched rows, plus the shared expert(s).
+ * MMOE page, "MoE++ expert layer" (heavy experts are standard MLPs) and
+ * "shared experts" (one dense expert always active). For bf16 the GEMMs
+ * run on tcgen05 tensor cores with TMEM accumulators fed by TMA; rows of
+ * an expert with no tokens, and the zero-computation experts, issue no
+ * MMA at all.
+ *   x_perm  [n_assign, d] rows grouped by `offsets` (from moe_dispatch)
+ *   W1      GELU: [n_heavy, h, d]; SwiGLU: [n_heavy, 2h, d] (gate rows, then up rows)
+ *   W2      [n_heavy, d, h]
+ *   x       [T, d], Ws1 [n_shared*h_shared, d], Ws2 [d, n_shared*h_shared]
+ *           (all three nullable when n_shared == 0)
+ *   y_perm  [n_assign, d] fp32 out: W2_e . act(W1_e . x_perm[r]) per row r
+ *   y_shared [T, d] fp32 out (nullable when n_shared == 0)
+ * Hidden activations are kept in `dtype` in the workspace.
+ */
+MOE_API int moe_grouped_mlp(const moe_config *cfg, const void *x_perm,
+                    const int32_t *offsets, const void *W1, const void *W2,
+                    const void *x, const void *Ws1, const void *Ws2,
+                    float *y_perm, float *y_shared, int32_t *dev_status,
+                    void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Combine back to token order, fused with the routing-weight scale and
+ * the residual add. DICE page, "Conditional Communication": the output of
+ * token i is the routing-score weighted sum of its experts' outputs.
+ *   y_s = r_s + y_shared[s] + sum over s's assignments a (in slot order) of
+ *         w[a] * { y_perm[row_of[a]] (heavy), x_s (identity), 0 (zero),
+ *                  const_vecs[c] (c-th constant expert) }
+ * summed in fp32 and rounded once to dtype.
+ *   sel, w       the selection (as in moe_dispatch) and its [n_assign] weights
+ *   row_of       from moe_dispatch;  tok_ptr/tok_assign: expert choice only
+ *   x            [T, d] (identity experts); const_vecs [n_const, d], nullable
+ *   residual     [T, d] nullable (r = 0);  y [T, d] out (dtype)
+ */
+MOE_API int moe_combine(const moe_config *cfg, const float *y_perm,
+                const float *y_shared, const int32_t *sel, const float *w,
+                const int32_t *row_of, const int32_t *tok_ptr,
+                const int32_t *tok_assign, const void *x,
+                const void *const_vecs, const void *residual, void *y,
+                int32_t *dev_status, moe_stream_t stream);
+
+/* Optional outputs of moe_forward (each pointer nullable; device memory). */
+typedef struct moe_forward_aux {
+  float *logits;     /* [T, E] fp32 */
+  float *probs;      /* [T, E] fp32 */
+  int32_t *sel;      /* [n_assign] idx (token choice, DES) or tok (expert choice) */
+  float *w;          /* [n_assign] fp32 routing weights */
+  int64_t *votes;    /* [E] DES-Vote only */
+  int32_t *core;     /* [M_core] DES-Vote only */
+  int32_t *offsets;  /* [n_heavy + 1] */
+} moe_forward_aux;
+
+/*
+ * The whole layer: router -> selection -> dispatch -> grouped MLP ->
+ * combine, every step a kernel of this library, all on `stream`, no host
+ * synchronisation (group sizes stay on the device).
+ *   x [T, d], residual [T, d] nullable, z_prev [T, E] fp32 nullable,
+ *   W_r [E, d], bias [E] fp32 nullable, W1, W2, Ws1, Ws2 as in
+ *   moe_grouped_mlp, const_vecs [n_const, d] nullable, y [T, d] out.
+ *   aux nullable: copies of the intermediate results for inspection.
+ */
+MOE_API int moe_forward(const moe_config *cfg, const void *x, const void *residual,
+                const float *z_prev, const void *W_r, const float *bias,
+                const void *W1, const void *W2, const void *Ws1,
+                const void *Ws2, const void *const_vecs, void *y,
+                const moe_forward_aux *aux, int32_t *dev_status, void *ws,
+                size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_forward with the activations in HOST memory: copies x_host (and
+ * residual_host, z_prev_host if given) to the device, runs the layer and
+ * copies y back to y_host, all enqueued on `stream`. Weights stay device
+ * pointers. For the copies to be asynchronous the host buffers should be
+ * pinned; the caller synchronises `stream` before reading y_host.
+ */
+MOE_API int moe_forward_host(const moe_config *cfg, const void *x_host,
+                     const void *residual_host, const float *z_prev_host,
+                     const void *W_r, const float *bias, const void *W1,
+                     const void *W2, const void *Ws1, const void *Ws2,
+                     const void *const_vecs, void *y_host,
+                     int32_t *dev_status, void *ws, size_t ws_bytes,
+                     moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

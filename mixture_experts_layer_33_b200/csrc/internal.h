@@ -1,0 +1,101 @@
+// Internal launch interface between the C ABI (moe_api.cu) and the kernel
+// translation units. Every launcher enqueues on `stream`, returns a
+// moe_status, and never synchronises the host.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+struct KindTable;
+
+#define MOE_CUDA_TRY(expr)                                   \
+  do {                                                       \
+    cudaError_t moe_err_ = (expr);                           \
+    if (moe_err_ != cudaSuccess) return MOE_ERR_CUDA;        \
+  } while (0)
+
+inline int last_launch_status() {
+  return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int num_sms();
+
+// router.cu: z = x W_r^T + bias + scale * z_prev; A = softmax(z); optional top-k.
+int launch_router(const void *x, const void *W_r, const float *bias,
+                  const float *z_prev, float z_prev_scale, int T, int d, int E,
+                  int dtype, float *logits, float *probs, int k, int renorm,
+                  int32_t *idx, float *w, cudaStream_t stream);
+int launch_select_topk(const float *logits, const float *probs, int T, int E,
+                       int k, int renorm, int32_t *idx, float *w,
+                       cudaStream_t stream);
+
+// select.cu: expert-choice radix select and the DES-Vote core set.
+int launch_expert_choice(const float *probs, int T, int E, int S, int C,
+                         int32_t *tok, float *w, cudaStream_t stream);
+int launch_des_vote(const float *probs, int N, int M, int K, int M_core,
+                    int64_t *votes, int32_t *core, int32_t *idx, float *w,
+                    cudaStream_t stream);
+
+// dispatch.cu
+struct DispatchArgs {
+  int routing;     // moe_routing
+  int T, E, n_heavy;
+  int k;           // token choice / DES: slots per token
+  int S, C;        // expert choice
+  int64_t n_assign;
+  const int32_t *sel;
+  int32_t *offsets, *perm, *row_of, *tok_ptr, *tok_assign;
+  int32_t *dev_status;
+};
+size_t dispatch_workspace_bytes(int64_t n_assign, int n_heavy);
+int launch_dispatch(const DispatchArgs &a, void *ws, cudaStream_t stream);
+int launch_gather_rows(const void *x, void *x_perm, const int32_t *perm,
+                       const int32_t *offsets, int n_heavy, int64_t max_rows,
+                       int d, int elem_bytes, cudaStream_t stream);
+
+// gemm_sm100.cu: grouped GEMM D = act(A . B^T) on tcgen05 (bf16 in, fp32 acc).
+enum GemmAct { kActNone = 0, kActGelu = 1, kActSwiglu = 2 };
+struct GemmProblem {
+  const void *A;        // [rows, K] bf16
+  int64_t a_rows;       // rows in the A tensor (TMA bound)
+  const void *B;        // [n_groups * b_rows_per_group, K] bf16
+  int b_rows_per_group; // N (none/GELU) or 2N (SwiGLU: gate rows then up rows)
+  int n_groups;
+  const int32_t *offsets;  // [n_groups + 1] device row offsets, or NULL: one group of a_rows rows
+  int N, K;
+  void *out;            // [rows, ld_out] (bf16 or fp32)
+  int64_t ld_out;
+};
+
+// Upper bound of the m-tiles of height bm over all groups of a problem.
+inline int64_t max_m_tiles(const GemmProblem &p, int bm) {
+  return (p.a_rows + bm - 1) / bm + (p.offsets ? p.n_groups : 0);
+}
+int launch_grouped_gemm_bf16(const GemmProblem *probs, int n_probs, int act,
+                             bool out_f32, int32_t *dev_status,
+                             cudaStream_t stream);
+
+// mlp_f32.cu: the same grouped GEMM in fp32 on CUDA cores (fp32 layers).
+int launch_grouped_gemm_f32(const GemmProblem &p, int act,
+                            cudaStream_t stream);
+
+// combine.cu
+struct CombineArgs {
+  int routing, T, d, E, k, S, C, dtype;
+  const float *y_perm, *y_shared;
+  const int32_t *sel;
+  const float *w;
+  const int32_t *row_of, *tok_ptr, *tok_assign;
+  const void *x, *const_vecs, *residual;
+  void *y;
+  int32_t *dev_status;
+};
+int launch_combine(const CombineArgs &a, const KindTable &kinds,
+                   cudaStream_t stream);
+
+}  // namespace moe

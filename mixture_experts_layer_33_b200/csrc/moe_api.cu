@@ -1,0 +1,467 @@
+// The C ABI of libmoe.so: argument checks, workspace layout and the
+// orchestration of the layer's kernels (declared in include/moe.h).
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int elem_bytes(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+
+int64_t n_assign_of(const moe_config &c) {
+  if (c.routing == MOE_EXPERT_CHOICE) return (int64_t)(c.T / c.group_size) * c.E * c.capacity;
+  return (int64_t)c.T * c.k;
+}
+
+int check_config(const moe_config *c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_BF16 && c->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d < 8 || c->d % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (c->E < 1 || c->E > 128) return c->E > 128 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (c->n_heavy < 0 || c->n_heavy > c->E) return MOE_ERR_INVALID_ARG;
+  if (c->n_heavy > 0 && (c->h < 8 || c->h % 8 != 0)) return MOE_ERR_INVALID_ARG;
+  if (c->act != MOE_GELU_ERF && c->act != MOE_SWIGLU) return MOE_ERR_INVALID_ARG;
+  for (int e = 0; e < c->E; ++e) {
+    int k = c->expert_kind[e];
+    if (e < c->n_heavy ? k != MOE_HEAVY : (k != MOE_IDENTITY && k != MOE_ZERO && k != MOE_CONST))
+      return MOE_ERR_INVALID_ARG;
+  }
+  if (c->n_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (c->n_shared > 0 && (c->h_shared < 8 || c->h_shared % 8 != 0)) return MOE_ERR_INVALID_ARG;
+  switch (c->routing) {
+    case MOE_TOKEN_TOPK:
+      if (c->k < 1 || c->k > c->E) return MOE_ERR_INVALID_ARG;
+      break;
+    case MOE_EXPERT_CHOICE:
+      if (c->group_size < 1 || c->T % c->group_size != 0) return MOE_ERR_INVALID_ARG;
+      if (c->capacity < 1 || c->capacity > c->group_size) return MOE_ERR_INVALID_ARG;
+      if (c->group_size > 16384) return MOE_ERR_UNSUPPORTED;
+      break;
+    case MOE_DES_VOTE:
+      if (c->k < 1 || c->k > c->M_core || c->M_core > c->E) return MOE_ERR_INVALID_ARG;
+      if (c->T > 4096) return MOE_ERR_UNSUPPORTED;
+      break;
+    default:
+      return MOE_ERR_INVALID_ARG;
+  }
+  if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_INVALID_ARG;
+  if (n_assign_of(*c) > (int64_t)0x7fffffff) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+KindTable kind_table(const moe_config &c) {
+  KindTable kt;
+  memset(&kt, 0, sizeof(kt));
+  int nc = 0;
+  for (int e = 0; e < c.E; ++e) {
+    kt.kind[e] = (int8_t)c.expert_kind[e];
+    kt.cidx[e] = (int16_t)(c.expert_kind[e] == MOE_CONST ? nc++ : 0);
+  }
+  return kt;
+}
+
+int n_const_of(const moe_config &c) {
+  int n = 0;
+  for (int e = 0; e < c.E; ++e) n += c.expert_kind[e] == MOE_CONST;
+  return n;
+}
+
+// Workspace layout shared by the entry points.
+struct Layout {
+  size_t logits, probs, sel, w, votes, core, offsets, perm, row_of, tok_ptr, tok_assign, dpart,
+      x_perm, H, H_sh, Y, Y_sh, x_dev, res_dev, zp_dev, y_dev, total;
+};
+
+Layout layout_of(const moe_config &c) {
+  Layout L;
+  const int64_t na = n_assign_of(c);
+  const size_t eb = elem_bytes(c.dtype);
+  const int64_t hs = (int64_t)c.n_shared * c.h_shared;
+  const int64_t h1 = c.h;  // hidden activations after the gate (SwiGLU halves 2h -> h)
+  size_t o = kAlign;  // the first slot is reserved, so a workspace is never empty
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  L.logits = take((size_t)c.T * c.E * 4);
+  L.probs = take((size_t)c.T * c.E * 4);
+  L.sel = take((size_t)na * 4);
+  L.w = take((size_t)na * 4);
+  L.votes = take((size_t)c.E * 8);
+  L.core = take((size_t)c.E * 4);
+  L.offsets = take((size_t)(c.n_heavy + 1) * 4);
+  L.perm = take((size_t)na * 4);
+  L.row_of = take((size_t)na * 4);
+  L.tok_ptr = take((size_t)(c.T + 1) * 4);
+  L.tok_assign = take((size_t)na * 4);
+  L.dpart = take(dispatch_workspace_bytes(na, c.n_heavy));
+  L.x_perm = take((size_t)na * c.d * eb);
+  L.H = take((size_t)na * h1 * eb);
+  L.H_sh = take((size_t)c.T * hs * eb);
+  L.Y = take((size_t)na * c.d * 4);
+  L.Y_sh = take(hs ? (size_t)c.T * c.d * 4 : 0);
+  L.x_dev = take((size_t)c.T * c.d * eb);
+  L.res_dev = take((size_t)c.T * c.d * eb);
+  L.zp_dev = take((size_t)c.T * c.E * 4);
+  L.y_dev = take((size_t)c.T * c.d * eb);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+int check_ws(const moe_config &c, void *ws, size_t ws_bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < layout_of(c).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offsets,
+                    const void *W1, const void *W2, const void *x, const void *Ws1,
+                    const void *Ws2, float *y_perm, float *y_shared, int32_t *dev_status,
+                    void *ws, const Layout &L, cudaStream_t stream) {
+  const int64_t na = n_assign_of(c);
+  const int64_t hs = (int64_t)c.n_shared * c.h_shared;
+  void *H = at<void>(ws, L.H);
+  void *H_sh = at<void>(ws, L.H_sh);
+  const int act1 = c.act == MOE_SWIGLU ? kActSwiglu : kActGelu;
+
+  GemmProblem g1r{}, g1s{}, g2r{}, g2s{};
+  g1r.A = x_perm; g1r.a_rows = na; g1r.B = W1; g1r.n_groups = c.n_heavy; g1r.offsets = offsets;
+  g1r.N = c.h; g1r.b_rows_per_group = act1 == kActSwiglu ? 2 * c.h : c.h; g1r.K = c.d;
+  g1r.out = H; g1r.ld_out = c.h;
+  g2r.A = H; g2r.a_rows = na; g2r.B = W2; g2r.n_groups = c.n_heavy; g2r.offsets = offsets;
+  g2r.N = c.d; g2r.b_rows_per_group = c.d; g2r.K = c.h; g2r.out = y_perm; g2r.ld_out = c.d;
+  g1s.A = x; g1s.a_rows = c.T; g1s.B = Ws1; g1s.n_groups = 1; g1s.offsets = nullptr;
+  g1s.N = (int)hs; g1s.b_rows_per_group = (int)hs; g1s.K = c.d; g1s.out = H_sh; g1s.ld_out = hs;
+  g2s.A = H_sh; g2s.a_rows = c.T; g2s.B = Ws2; g2s.n_groups = 1; g2s.offsets = nullptr;
+  g2s.N = c.d; g2s.b_rows_per_group = c.d; g2s.K = (int)hs; g2s.out = y_shared; g2s.ld_out = c.d;
+  const bool routed = c.n_heavy > 0 && na > 0;
+  const bool shared = hs > 0 && c.T > 0;
+
+  int st = MOE_OK;
+  if (c.dtype == MOE_BF16) {
+    // GEMM1 (+activation): routed and shared in one tile stream when they share the activation.
+    if (routed && shared && act1 == kActGelu) {
+      GemmProblem p1[2] = {g1r, g1s};
+      st = launch_grouped_gemm_bf16(p1, 2, kActGelu, false, dev_status, stream);
+    } else {
+      if (routed) st = launch_grouped_gemm_bf16(&g1r, 1, act1, false, dev_status, stream);
+      if (st == MOE_OK && shared) st = launch_grouped_gemm_bf16(&g1s, 1, kActGelu, false, dev_status, stream);
+    }
+    if (st != MOE_OK) return st;
+    // GEMM2: the longer-K shared problem first so the tile stream ends on short tiles.
+    if (routed && shared) {
+      GemmProblem p2[2] = {g2s, g2r};
+      st = launch_grouped_gemm_bf16(p2, 2, kActNone, true, dev_status, stream);
+    } else if (routed) {
+      st = launch_grouped_gemm_bf16(&g2r, 1, kActNone, true, dev_status, stream);
+    } else if (shared) {
+      st = launch_grouped_gemm_bf16(&g2s, 1, kActNone, true, dev_status, stream);
+    }
+    return st;
+  }
+  if (routed) {
+    st = launch_grouped_gemm_f32(g1r, act1, stream);
+    if (st == MOE_OK) st = launch_grouped_gemm_f32(g2r, kActNone, stream);
+  }
+  if (st == MOE_OK && shared) {
+    st = launch_grouped_gemm_f32(g1s, kActGelu, stream);
+    if (st == MOE_OK) st = launch_grouped_gemm_f32(g2s, kActNone, stream);
+  }
+  return st;
+}
+
+DispatchArgs dispatch_args(const moe_config &c, const int32_t *sel, int32_t *offsets,
+                           int32_t *perm, int32_t *row_of, int32_t *tok_ptr,
+                           int32_t *tok_assign, int32_t *dev_status) {
+  DispatchArgs a;
+  a.routing = c.routing;
+  a.T = c.T; a.E = c.E; a.n_heavy = c.n_heavy; a.k = c.k;
+  a.S = c.group_size; a.C = c.capacity;
+  a.n_assign = n_assign_of(c);
+  a.sel = sel; a.offsets = offsets; a.perm = perm; a.row_of = row_of;
+  a.tok_ptr = tok_ptr; a.tok_assign = tok_assign; a.dev_status = dev_status;
+  return a;
+}
+
+CombineArgs combine_args(const moe_config &c, const float *y_perm, const float *y_shared,
+                         const int32_t *sel, const float *w, const int32_t *row_of,
+                         const int32_t *tok_ptr, const int32_t *tok_assign, const void *x,
+                         const void *const_vecs, const void *residual, void *y,
+                         int32_t *dev_status) {
+  CombineArgs a;
+  a.routing = c.routing; a.T = c.T; a.d = c.d; a.E = c.E; a.k = c.k;
+  a.S = c.group_size; a.C = c.capacity; a.dtype = c.dtype;
+  a.y_perm = y_perm; a.y_shared = y_shared; a.sel = sel; a.w = w; a.row_of = row_of;
+  a.tok_ptr = tok_ptr; a.tok_assign = tok_assign; a.x = x; a.const_vecs = const_vecs;
+  a.residual = residual; a.y = y; a.dev_status = dev_status;
+  return a;
+}
+
+int forward_device(const moe_config &c, const void *x, const void *residual,
+                   const float *z_prev, const void *W_r, const float *bias, const void *W1,
+                   const void *W2, const void *Ws1, const void *Ws2, const void *const_vecs,
+                   void *y, const moe_forward_aux *aux, int32_t *dev_status, void *ws,
+                   const Layout &L, cudaStream_t stream) {
+  float *logits = (aux && aux->logits) ? aux->logits : at<float>(ws, L.logits);
+  float *probs = (aux && aux->probs) ? aux->probs : at<float>(ws, L.probs);
+  int32_t *sel = (aux && aux->sel) ? aux->sel : at<int32_t>(ws, L.sel);
+  float *w = (aux && aux->w) ? aux->w : at<float>(ws, L.w);
+  int64_t *votes = (aux && aux->votes) ? aux->votes : at<int64_t>(ws, L.votes);
+  int32_t *core = (aux && aux->core) ? aux->core : at<int32_t>(ws, L.core);
+  int32_t *offsets = (aux && aux->offsets) ? aux->offsets : at<int32_t>(ws, L.offsets);
+  int32_t *perm = at<int32_t>(ws, L.perm), *row_of = at<int32_t>(ws, L.row_of);
+  int32_t *tok_ptr = at<int32_t>(ws, L.tok_ptr), *tok_assign = at<int32_t>(ws, L.tok_assign);
+  const int64_t na = n_assign_of(c);
+  const int64_t hs = (int64_t)c.n_shared * c.h_shared;
+  float *Y = at<float>(ws, L.Y);
+  float *Y_sh = hs ? at<float>(ws, L.Y_sh) : nullptr;
+  void *x_perm = at<void>(ws, L.x_perm);
+
+  int st = launch_router(x, W_r, bias, z_prev, c.gate_residual_scale, c.T, c.d, c.E, c.dtype,
+                         logits, probs, c.routing == MOE_TOKEN_TOPK ? c.k : 0, c.renorm, sel, w,
+                         stream);
+  if (st != MOE_OK) return st;
+  if (c.routing == MOE_EXPERT_CHOICE)
+    st = launch_expert_choice(probs, c.T, c.E, c.group_size, c.capacity, sel, w, stream);
+  else if (c.routing == MOE_DES_VOTE)
+    st = launch_des_vote(probs, c.T, c.E, c.k, c.M_core, votes, core, sel, w, stream);
+  if (st != MOE_OK) return st;
+
+  DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
+  st = launch_dispatch(da, at<void>(ws, L.dpart), stream);
+  if (st != MOE_OK) return st;
+  if (c.n_heavy > 0) {
+    st = launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, na, c.d, elem_bytes(c.dtype), stream);
+    if (st != MOE_OK) return st;
+  }
+  st = run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, Y, Y_sh, dev_status, ws, L, stream);
+  if (st != MOE_OK) return st;
+  CombineArgs ca = combine_args(c, Y, Y_sh, sel, w, row_of, tok_ptr, tok_assign, x, const_vecs,
+                                residual, y, dev_status);
+  return launch_combine(ca, kind_table(c), stream);
+}
+
+int check_forward_ptrs(const moe_config &c, const void *x, const void *W_r, const void *W1,
+                       const void *W2, const void *Ws1, const void *Ws2,
+                       const void *const_vecs, const void *y) {
+  if (!W_r || !aligned16(W_r)) return MOE_ERR_INVALID_ARG;
+  if (c.T > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  if (c.n_heavy > 0 && (!W1 || !W2 || !aligned16(W1) || !aligned16(W2))) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!Ws1 || !Ws2 || !aligned16(Ws1) || !aligned16(Ws2))) return MOE_ERR_INVALID_ARG;
+  if (n_const_of(c) > 0 && (!const_vecs || !aligned16(const_vecs))) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: valid but unsupported";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call failed";
+    case MOE_ERR_DEVICE_STATUS: return "MOE_ERR_DEVICE_STATUS: device status word set";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: bounded device wait expired";
+    default: return "unknown moe_status";
+  }
+}
+
+int moe_device_check(int device) {
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return (major == 10 && minor == 0) ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+int moe_num_assignments(const moe_config *cfg, int64_t *n_assign) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!n_assign) return MOE_ERR_INVALID_ARG;
+  *n_assign = n_assign_of(*cfg);
+  return MOE_OK;
+}
+
+int moe_workspace_size(const moe_config *cfg, size_t *bytes) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = layout_of(*cfg).total;
+  return MOE_OK;
+}
+
+int moe_router(const void *x, const void *W_r, const float *bias, const float *z_prev,
+               float z_prev_scale, int T, int d, int E, int dtype, float *logits, float *probs,
+               int k, int renorm, int32_t *idx, float *w, moe_stream_t stream) {
+  if (T < 0 || d < 8 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (E > 128) return MOE_ERR_UNSUPPORTED;
+  if (dtype != MOE_BF16 && dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_BF16 && d % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (!W_r) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !logits || !probs)) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_BF16 && (!aligned16(x) || !aligned16(W_r))) return MOE_ERR_INVALID_ARG;
+  if (k < 0 || k > E || (k > 0 && (!idx || !w))) return MOE_ERR_INVALID_ARG;
+  if (renorm != 0 && renorm != 1) return MOE_ERR_INVALID_ARG;
+  return launch_router(x, W_r, bias, z_prev, z_prev_scale, T, d, E, dtype, logits, probs, k,
+                       renorm, idx, w, stream);
+}
+
+int moe_select_topk(const float *logits, const float *probs, int T, int E, int k, int renorm,
+                    int32_t *idx, float *w, moe_stream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > 128) return MOE_ERR_UNSUPPORTED;
+  if (!logits || !probs || !idx || !w) return MOE_ERR_INVALID_ARG;
+  if (renorm != 0 && renorm != 1) return MOE_ERR_INVALID_ARG;
+  return launch_select_topk(logits, probs, T, E, k, renorm, idx, w, stream);
+}
+
+int moe_select_expert_choice(const float *probs, int T, int E, int group_size, int C,
+                             int32_t *tok, float *w, moe_stream_t stream) {
+  if (T < 0 || E < 1 || group_size < 1 || T % group_size != 0) return MOE_ERR_INVALID_ARG;
+  if (C < 1 || C > group_size) return MOE_ERR_INVALID_ARG;
+  if (group_size > 16384) return MOE_ERR_UNSUPPORTED;
+  if (!probs || !tok || !w) return MOE_ERR_INVALID_ARG;
+  return launch_expert_choice(probs, T, E, group_size, C, tok, w, stream);
+}
+
+int moe_core_set_vote(const float *probs, int N, int M, int K, int M_core, int64_t *votes,
+                      int32_t *core, int32_t *idx, float *w, moe_stream_t stream) {
+  if (N < 0 || M < 1 || K < 1 || K > M_core || M_core > M) return MOE_ERR_INVALID_ARG;
+  if (M > MOE_MAX_EXPERTS || N > 4096) return MOE_ERR_UNSUPPORTED;
+  if (!probs || !votes || !core || !idx || !w) return MOE_ERR_INVALID_ARG;
+  return launch_des_vote(probs, N, M, K, M_core, votes, core, idx, w, stream);
+}
+
+int moe_dispatch(const moe_config *cfg, const int32_t *sel, const void *x, void *x_perm,
+                 int32_t *offsets, int32_t *perm, int32_t *row_of, int32_t *tok_ptr,
+                 int32_t *tok_assign, int32_t *dev_status, void *ws, size_t ws_bytes,
+                 moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  if (n_assign_of(c) > 0 && (!sel || !perm || !row_of)) return MOE_ERR_INVALID_ARG;
+  if (x_perm && (!x || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (c.routing == MOE_EXPERT_CHOICE && (!tok_ptr != !tok_assign)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const Layout L = layout_of(c);
+  DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
+  st = launch_dispatch(da, at<void>(ws, L.dpart), stream);
+  if (st != MOE_OK || !x_perm || c.n_heavy == 0) return st;
+  return launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, n_assign_of(c), c.d,
+                            elem_bytes(c.dtype), stream);
+}
+
+int moe_grouped_mlp(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                    const void *W1, const void *W2, const void *x, const void *Ws1,
+                    const void *Ws2, float *y_perm, float *y_shared, int32_t *dev_status,
+                    void *ws, size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (c.n_heavy > 0 && (!x_perm || !offsets || !W1 || !W2 || !y_perm)) return MOE_ERR_INVALID_ARG;
+  if (c.n_heavy > 0 && (!aligned16(x_perm) || !aligned16(W1) || !aligned16(W2) || !aligned16(y_perm)))
+    return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!x || !Ws1 || !Ws2 || !y_shared)) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && (!aligned16(x) || !aligned16(Ws1) || !aligned16(Ws2) || !aligned16(y_shared)))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  return run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, y_perm, y_shared, dev_status,
+                         ws, layout_of(c), stream);
+}
+
+int moe_combine(const moe_config *cfg, const float *y_perm, const float *y_shared,
+                const int32_t *sel, const float *w, const int32_t *row_of,
+                const int32_t *tok_ptr, const int32_t *tok_assign, const void *x,
+                const void *const_vecs, const void *residual, void *y, int32_t *dev_status,
+                moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (c.T > 0 && (!sel || !w || !row_of || !x || !y)) return MOE_ERR_INVALID_ARG;
+  if (c.n_heavy > 0 && !y_perm) return MOE_ERR_INVALID_ARG;
+  if (c.n_shared > 0 && !y_shared) return MOE_ERR_INVALID_ARG;
+  if (c.routing == MOE_EXPERT_CHOICE && (!tok_ptr || !tok_assign)) return MOE_ERR_INVALID_ARG;
+  if (n_const_of(c) > 0 && !const_vecs) return MOE_ERR_INVALID_ARG;
+  const void *ptrs[6] = {y_perm, y_shared, x, const_vecs, residual, y};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  CombineArgs ca = combine_args(c, y_perm, c.n_shared > 0 ? y_shared : nullptr, sel, w, row_of,
+                                tok_ptr, tok_assign, x, const_vecs, residual, y, dev_status);
+  return launch_combine(ca, kind_table(c), stream);
+}
+
+int moe_forward(const moe_config *cfg, const void *x, const void *residual, const float *z_prev,
+                const void *W_r, const float *bias, const void *W1, const void *W2,
+                const void *Ws1, const void *Ws2, const void *const_vecs, void *y,
+                const moe_forward_aux *aux, int32_t *dev_status, void *ws, size_t ws_bytes,
+                moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if ((st = check_forward_ptrs(c, x, W_r, W1, W2, Ws1, Ws2, const_vecs, y)) != MOE_OK) return st;
+  if (residual && !aligned16(residual)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  return forward_device(c, x, residual, z_prev, W_r, bias, W1, W2, Ws1, Ws2, const_vecs, y, aux,
+                        dev_status, ws, layout_of(c), stream);
+}
+
+int moe_forward_host(const moe_config *cfg, const void *x_host, const void *residual_host,
+                     const float *z_prev_host, const void *W_r, const float *bias,
+                     const void *W1, const void *W2, const void *Ws1, const void *Ws2,
+                     const void *const_vecs, void *y_host, int32_t *dev_status, void *ws,
+                     size_t ws_bytes, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (c.T > 0 && (!x_host || !y_host)) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(c, ws, ws_bytes)) != MOE_OK) return st;
+  const Layout L = layout_of(c);
+  void *xd = at<void>(ws, L.x_dev), *yd = at<void>(ws, L.y_dev);
+  if ((st = check_forward_ptrs(c, xd, W_r, W1, W2, Ws1, Ws2, const_vecs, yd)) != MOE_OK) return st;
+  const size_t act_bytes = (size_t)c.T * c.d * elem_bytes(c.dtype);
+  if (act_bytes) MOE_CUDA_TRY(cudaMemcpyAsync(xd, x_host, act_bytes, cudaMemcpyHostToDevice, stream));
+  const void *rd = nullptr;
+  if (residual_host == x_host) {
+    rd = xd;
+  } else if (residual_host && act_bytes) {
+    void *r = at<void>(ws, L.res_dev);
+    MOE_CUDA_TRY(cudaMemcpyAsync(r, residual_host, act_bytes, cudaMemcpyHostToDevice, stream));
+    rd = r;
+  }
+  const float *zd = nullptr;
+  if (z_prev_host && c.T > 0) {
+    float *z = at<float>(ws, L.zp_dev);
+    MOE_CUDA_TRY(cudaMemcpyAsync(z, z_prev_host, (size_t)c.T * c.E * 4, cudaMemcpyHostToDevice, stream));
+    zd = z;
+  }
+  st = forward_device(c, xd, rd, zd, W_r, bias, W1, W2, Ws1, Ws2, const_vecs, yd, nullptr,
+                      dev_status, ws, L, stream);
+  if (st != MOE_OK) return st;
+  if (act_bytes) MOE_CUDA_TRY(cudaMemcpyAsync(y_host, yd, act_bytes, cudaMemcpyDeviceToHost, stream));
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,346 @@
+// Router GEMM + softmax + token-choice top-k, fused (one kernel).
+//
+// EC-DiT: Scaling Diffusion Transformers with Adaptive Expert-Choice
+// Routing, section 3 "Expert-Choice routing formula": the affinity of token
+// s to expert i is the softmax over the E experts of (x' W_r)_{s,i}.
+// MMOE: Modernizing Diffusion Transformers with Efficient Expert Design,
+// "gate-residual routing": the previous expert layer's gate logits are
+// added to the router logits (z = x W_r + b + scale * z_prev).
+// EC-DiT section 3 "Token-Choice routing": each token keeps its top-k
+// experts.
+//
+// bf16 path: a CTA owns 64 tokens; its 4 warps each run m16n8k16 bf16
+// tensor-core MMAs (fp32 accumulate) over cp.async-staged tiles of x and
+// W_r, so x is read from HBM exactly once. The N dimension of this GEMM is
+// E <= 128, far too narrow for a 128-wide tcgen05 tile; the kernel is bound
+// by reading x. The logits tile is then parked in shared memory and each
+// warp finishes its 16 tokens with warp-shuffle softmax and warp-shuffle
+// argmax rounds for the top-k (ties to the lower expert id).
+// fp32 path: plain FMA dot products, one warp per token (fp32 layers are
+// small and must stay exact to fp32 rounding).
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kBM = 64;        // tokens per CTA
+constexpr int kBK = 64;        // model-width slice per pipeline stage
+constexpr int kLDS = kBK + 8;  // padded smem row (bf16): conflict-free ldmatrix
+constexpr int kStages = 3;
+constexpr int kThreads = 128;
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  int n = valid ? 16 : 0;  // 0 bytes read: the 16 smem bytes are zero-filled
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *p) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(s));
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[2], const void *p) {
+  uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r[0]), "=r"(r[1]) : "r"(s));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4],
+                                               const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Softmax of one token row held by a warp: expert e = lane + 32*v.
+template <int VPL>
+__device__ __forceinline__ void row_softmax(const float (&z)[VPL], int E, float (&A)[VPL]) {
+  const int lane = threadIdx.x & 31;
+  float m = -INFINITY;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v)
+    if (lane + 32 * v < E) m = fmaxf(m, z[v]);
+  m = warp_max(m);
+  float s = 0.f;
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    A[v] = (lane + 32 * v < E) ? expf(z[v] - m) : 0.f;
+    s += A[v];
+  }
+  s = warp_sum(s);
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) A[v] = A[v] / s;
+}
+
+// Top-k of one token row held by a warp, ranked by z, ties to the lower id.
+// Lane 0 writes idx_row[0..k) in rank order and w_row = A (or A / sum).
+template <int VPL>
+__device__ __forceinline__ void row_topk(const float (&z)[VPL], const float (&A)[VPL], int E,
+                                         int k, int renorm, int32_t *idx_row, float *w_row) {
+  const int lane = threadIdx.x & 31;
+  bool taken[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) taken[v] = false;
+  float wsum = 0.f;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      int e = lane + 32 * v;
+      if (e < E && !taken[v] && better(z[v], e, bv, bi)) { bv = z[v]; bi = e; }
+    }
+    warp_argmax(bv, bi);
+    float a_own = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+      if (lane + 32 * v == bi) { taken[v] = true; a_own = A[v]; }
+    float a = __shfl_sync(0xffffffffu, a_own, bi & 31);
+    wsum += a;
+    if (lane == 0) {
+      idx_row[r] = bi;
+      w_row[r] = a;
+    }
+  }
+  if (renorm && lane == 0)
+    for (int r = 0; r < k; ++r) w_row[r] = w_row[r] / wsum;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads)
+router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Wr,
+                   const float *__restrict__ bias, const float *__restrict__ zprev, float zscale,
+                   int T, int d, int E, float *__restrict__ logits, float *__restrict__ probs,
+                   int k, int renorm, int32_t *__restrict__ idx, float *__restrict__ w) {
+  constexpr int EP = NT * 8;
+  constexpr int VPL = (EP + 31) / 32;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __nv_bfloat16 *sX = reinterpret_cast<__nv_bfloat16 *>(smem_raw);   // [stages][kBM][kLDS]
+  __nv_bfloat16 *sW = sX + kStages * kBM * kLDS;                      // [stages][EP][kLDS]
+  float *sZ = reinterpret_cast<float *>(sW + kStages * EP * kLDS);    // [kBM][EP + 1]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * kBM;
+  const int nk = (d + kBK - 1) / kBK;
+
+  auto load_stage = [&](int stage, int kb) {
+    const int k0 = kb * kBK;
+    for (int c = tid; c < kBM * (kBK / 8); c += kThreads) {
+      int r = c >> 3, cc = c & 7, gr = t0 + r, gk = k0 + cc * 8;
+      bool ok = gr < T && gk < d;
+      const __nv_bfloat16 *src = x + (size_t)(ok ? gr : 0) * d + (ok ? gk : 0);
+      cp_async16(sX + (stage * kBM + r) * kLDS + cc * 8, src, ok);
+    }
+    for (int c = tid; c < EP * (kBK / 8); c += kThreads) {
+      int r = c >> 3, cc = c & 7, gk = k0 + cc * 8;
+      bool ok = r < E && gk < d;
+      const __nv_bfloat16 *src = Wr + (size_t)(ok ? r : 0) * d + (ok ? gk : 0);
+      cp_async16(sW + (stage * EP + r) * kLDS + cc * 8, src, ok);
+    }
+  };
+
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < nk) load_stage(s, s);
+    cp_async_commit();
+  }
+
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+
+  for (int kb = 0; kb < nk; ++kb) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();
+    {
+      int nkb = kb + kStages - 1;
+      if (nkb < nk) load_stage(nkb % kStages, nkb);
+      cp_async_commit();
+    }
+    const int st = kb % kStages;
+    const __nv_bfloat16 *tX = sX + (st * kBM + warp * 16) * kLDS;
+    const __nv_bfloat16 *tW = sW + st * EP * kLDS;
+#pragma unroll
+    for (int kk = 0; kk < kBK / 16; ++kk) {
+      uint32_t a[4];
+      ldmatrix_x4(a, tX + (lane & 15) * kLDS + kk * 16 + (lane >> 4) * 8);
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        uint32_t b[2];
+        ldmatrix_x2(b, tW + (n * 8 + (lane & 7)) * kLDS + kk * 16 + ((lane >> 3) & 1) * 8);
+        mma_bf16_16816(acc[n], a, b);
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  // Park the 64 x EP logits tile in shared memory.
+  {
+    const int r0 = warp * 16 + (lane >> 2);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int c0 = n * 8 + (lane & 3) * 2;
+      sZ[r0 * (EP + 1) + c0] = acc[n][0];
+      sZ[r0 * (EP + 1) + c0 + 1] = acc[n][1];
+      sZ[(r0 + 8) * (EP + 1) + c0] = acc[n][2];
+      sZ[(r0 + 8) * (EP + 1) + c0 + 1] = acc[n][3];
+    }
+  }
+  __syncthreads();
+
+  for (int i = 0; i < 16; ++i) {
+    const int r = warp * 16 + i, s = t0 + r;
+    if (s >= T) break;
+    float z[VPL], A[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      int e = lane + 32 * v;
+      float zz = -INFINITY;
+      if (e < E) {
+        zz = sZ[r * (EP + 1) + e];
+        if (bias) zz += bias[e];
+        if (zprev) zz += zscale * zprev[(size_t)s * E + e];
+        logits[(size_t)s * E + e] = zz;
+      }
+      z[v] = zz;
+    }
+    row_softmax<VPL>(z, E, A);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      int e = lane + 32 * v;
+      if (e < E) probs[(size_t)s * E + e] = A[v];
+    }
+    if (k > 0) row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
+  }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(kThreads)
+router_f32_kernel(const float *__restrict__ x, const float *__restrict__ Wr,
+                  const float *__restrict__ bias, const float *__restrict__ zprev, float zscale,
+                  int T, int d, int E, float *__restrict__ logits, float *__restrict__ probs,
+                  int k, int renorm, int32_t *__restrict__ idx, float *__restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int s = gw; s < T; s += nw) {
+    const float *xr = x + (size_t)s * d;
+    float z[VPL], A[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) z[v] = -INFINITY;
+    for (int e = 0; e < E; ++e) {
+      const float *wr = Wr + (size_t)e * d;
+      float p = 0.f;
+      for (int j = lane; j < d; j += 32) p = fmaf(xr[j], wr[j], p);
+      p = warp_sum(p);
+      if (bias) p += bias[e];
+      if (zprev) p += zscale * zprev[(size_t)s * E + e];
+#pragma unroll
+      for (int v = 0; v < VPL; ++v)
+        if (lane + 32 * v == e) z[v] = p;
+    }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      int e = lane + 32 * v;
+      if (e < E) logits[(size_t)s * E + e] = z[v];
+    }
+    row_softmax<VPL>(z, E, A);
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      int e = lane + 32 * v;
+      if (e < E) probs[(size_t)s * E + e] = A[v];
+    }
+    if (k > 0) row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
+  }
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(kThreads)
+select_topk_kernel(const float *__restrict__ logits, const float *__restrict__ probs, int T,
+                   int E, int k, int renorm, int32_t *__restrict__ idx, float *__restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int s = gw; s < T; s += nw) {
+    float z[VPL], A[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      int e = lane + 32 * v;
+      z[v] = e < E ? logits[(size_t)s * E + e] : -INFINITY;
+      A[v] = e < E ? probs[(size_t)s * E + e] : 0.f;
+    }
+    row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
+  }
+}
+
+template <int NT>
+int run_router_bf16(const void *x, const void *Wr, const float *bias, const float *zprev,
+                    float zscale, int T, int d, int E, float *logits, float *probs, int k,
+                    int renorm, int32_t *idx, float *w, cudaStream_t stream) {
+  constexpr int EP = NT * 8;
+  const size_t smem = (size_t)kStages * (kBM + EP) * kLDS * sizeof(__nv_bfloat16) +
+                      (size_t)kBM * (EP + 1) * sizeof(float);
+  auto kern = router_bf16_kernel<NT>;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  dim3 grid((T + kBM - 1) / kBM);
+  kern<<<grid, kThreads, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x),
+                                         static_cast<const __nv_bfloat16 *>(Wr), bias, zprev,
+                                         zscale, T, d, E, logits, probs, k, renorm, idx, w);
+  return last_launch_status();
+}
+
+int warp_grid(int rows) {
+  int warps_per_block = kThreads / 32;
+  int blocks = (rows + warps_per_block - 1) / warps_per_block;
+  int cap = num_sms() * 16;
+  return blocks < cap ? blocks : cap;
+}
+
+}  // namespace
+
+int launch_router(const void *x, const void *W_r, const float *bias, const float *z_prev,
+                  float z_prev_scale, int T, int d, int E, int dtype, float *logits,
+                  float *probs, int k, int renorm, int32_t *idx, float *w,
+                  cudaStream_t stream) {
+  if (T == 0) return MOE_OK;
+  if (dtype == MOE_BF16) {
+    const int nt = (E + 7) / 8;
+    if (nt <= 1) return run_router_bf16<1>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, stream);
+    if (nt <= 2) return run_router_bf16<2>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, stream);
+    if (nt <= 3) return run_router_bf16<3>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, stream);
+    if (nt <= 4) return run_router_bf16<4>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, stream);
+    if (nt <= 8) return run_router_bf16<8>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, stream);
+    return run_router_bf16<16>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, stream);
+  }
+  const float *xf = static_cast<const float *>(x);
+  const float *wf = static_cast<const float *>(W_r);
+  const int grid = warp_grid(T);
+  const int vpl = (E + 31) / 32;
+  if (vpl == 1) router_f32_kernel<1><<<grid, kThreads, 0, stream>>>(xf, wf, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
+  else if (vpl == 2) router_f32_kernel<2><<<grid, kThreads, 0, stream>>>(xf, wf, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
+  else router_f32_kernel<4><<<grid, kThreads, 0, stream>>>(xf, wf, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
+  return last_launch_status();
+}
+
+int launch_select_topk(const float *logits, const float *probs, int T, int E, int k,
+                       int renorm, int32_t *idx, float *w, cudaStream_t stream) {
+  if (T == 0) return MOE_OK;
+  const int grid = warp_grid(T);
+  const int vpl = (E + 31) / 32;
+  if (vpl == 1) select_topk_kernel<1><<<grid, kThreads, 0, stream>>>(logits, probs, T, E, k, renorm, idx, w);
+  else if (vpl == 2) select_topk_kernel<2><<<grid, kThreads, 0, stream>>>(logits, probs, T, E, k, renorm, idx, w);
+  else select_topk_kernel<4><<<grid, kThreads, 0, stream>>>(logits, probs, T, E, k, renorm, idx, w);
+  return last_launch_status();
+}
+
+}  // namespace moe

@@ -1,0 +1,254 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small cases run the whole oracle and span several 128-row tiles with
+ragged tails; the full workloads compare the router and every selection
+index in full and the layer output on a seeded sample of tokens (the
+oracle computes each sampled token's output exactly). Selection, dispatch
+and core-set indices must be bit-identical with the oracle fed the GPU's
+own fp32 logits/affinities; the router within 1e-4, the layer within 2e-2
+(bf16) or 1e-4 (fp32), all normwise relative.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_33_b200 import inputs as gen
+from tests import parity_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    ("tiny_fp32", {}),
+    ("ditmoe_xl", dict(T=600, d=256, h=512, h_shared=256)),
+    ("ecdit", dict(T=6 * 64, group_size=64, d=256, E=16, h=512, capacity=8)),
+    ("des_vote", dict(d=256, h=256)),
+    ("mmoe", dict(T=600, d=256, h=512, h_shared=256)),
+    ("mmoe_skewed", dict(T=600, d=256, h=512, h_shared=256)),
+]
+FULL = ["tiny_fp32", "ditmoe_xl", "ecdit", "des_vote", "mmoe", "mmoe_skewed"]
+
+
+def _check_router(cfg, hin, out):
+    z_ref = oracle.router_logits(hin["x"], hin["W_r"], hin["logit_bias"], hin["z_prev"],
+                                 cfg["gate_residual_scale"])
+    assert H.normwise(out["logits"], z_ref) <= H.ROUTER_TOL
+    A = out["probs"].astype(np.float64)
+    assert np.all(A >= 0)
+    assert np.max(np.abs(A.sum(axis=1) - 1.0)) <= H.ROWSUM_TOL
+    assert H.normwise(A, oracle.softmax_rows(z_ref)) <= H.ROUTER_TOL
+    return z_ref
+
+
+def _check_selection(cfg, out):
+    gpu = H.selection_of(cfg, out)
+    ref = H.oracle_selection_from_gpu(cfg, out)
+    key = "tok" if cfg["routing"] == "expert_choice" else "idx"
+    np.testing.assert_array_equal(gpu[key], ref[key])
+    np.testing.assert_array_equal(gpu["w"].astype(np.float64), ref["w"])
+    if cfg["routing"] == "des_vote":
+        np.testing.assert_array_equal(out["votes"], ref["votes"])
+        np.testing.assert_array_equal(out["core"][:cfg["M_core"]], ref["core"])
+    a_tok, a_exp, _ = oracle.assignments_from_selection(cfg, gpu)
+    offsets, *_ = oracle.dispatch(a_tok, a_exp, cfg["E_heavy"], cfg["T"])
+    np.testing.assert_array_equal(out["offsets"], offsets)
+    return gpu
+
+
+@pytest.mark.parametrize("name,over", SMALL, ids=[s[0] for s in SMALL])
+def test_layer_small_full_oracle(name, over):
+    cfg = gen.workload(name, **over)
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    assert out["status"] == 0
+    hin = H.host(inp)
+    _check_router(cfg, hin, out)
+    sel = _check_selection(cfg, out)
+    y_ref = H.oracle_layer(cfg, hin, sel)
+    assert H.normwise(out["y"], y_ref) <= H.Y_TOL[cfg["dtype"]]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_layer_full_size_sampled(name):
+    cfg = gen.workload(name)
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    assert out["status"] == 0
+    hin = H.host(inp)
+    _check_router(cfg, hin, out)
+    sel = _check_selection(cfg, out)
+    rng = np.random.default_rng(1234)
+    T = cfg["T"]
+    tokens = np.sort(rng.choice(T, size=min(T, 192), replace=False))
+    tokens[-1] = T - 1  # include the ragged end of the last tile
+    y_ref = H.oracle_layer(cfg, hin, sel, tokens=tokens)
+    assert H.normwise(out["y"][tokens], y_ref) <= H.Y_TOL[cfg["dtype"]]
+
+
+@pytest.mark.parametrize("name", ["ditmoe_xl", "mmoe"])
+def test_independent_routing_flips_are_near_ties(name):
+    # The oracle routes from its own fp64 logits; any set that differs from
+    # the GPU's must be a near tie of the ranking key.
+    cfg = gen.workload(name)
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    hin = H.host(inp)
+    z_ref = oracle.router_logits(hin["x"], hin["W_r"], hin["logit_bias"], hin["z_prev"],
+                                 cfg["gate_residual_scale"])
+    idx_ref = oracle.topk_token_choice(z_ref, cfg["k"])
+    idx_gpu = out["sel"].reshape(cfg["T"], cfg["k"])
+    scale = np.max(np.abs(z_ref))
+    for s in np.nonzero(np.any(np.sort(idx_ref, 1) != np.sort(idx_gpu, 1), axis=1))[0]:
+        kth_ref = z_ref[s, idx_ref[s, -1]]
+        gpu_min = z_ref[s, idx_gpu[s]].min()
+        assert abs(kth_ref - gpu_min) <= 1e-5 * scale
+
+
+@pytest.mark.parametrize("name,over", SMALL[1:4], ids=[s[0] for s in SMALL[1:4]])
+def test_stagewise_entry_points(name, over):
+    """Each entry point alone: router -> select -> dispatch -> grouped MLP -> combine."""
+    m = H.moe()
+    cfg = gen.workload(name, **over)
+    inp = gen.make_inputs(cfg, "cuda")
+    hin = H.host(inp)
+    c = m.make_config(cfg)
+    na = m.num_assignments(c)
+    T, E, d = cfg["T"], cfg["E"], cfg["d"]
+    dev = "cuda"
+    logits = torch.empty(T, E, device=dev)
+    probs = torch.empty(T, E, device=dev)
+    sel = torch.empty(na, dtype=torch.int32, device=dev)
+    w = torch.empty(na, device=dev)
+    r = cfg["routing"]
+    m.router(inp["x"], inp["W_r"], logits, probs, bias=inp["logit_bias"], z_prev=inp["z_prev"],
+             z_prev_scale=cfg["gate_residual_scale"], k=cfg["k"] if r == "token_topk" else 0,
+             idx=sel if r == "token_topk" else None, w=w if r == "token_topk" else None)
+    if r == "expert_choice":
+        m.select_expert_choice(probs, cfg["group_size"], cfg["capacity"], sel, w)
+    elif r == "des_vote":
+        votes = torch.empty(E, dtype=torch.int64, device=dev)
+        core = torch.empty(cfg["M_core"], dtype=torch.int32, device=dev)
+        m.core_set_vote(probs, cfg["k"], cfg["M_core"], votes, core, sel, w)
+    else:
+        # the standalone selection must agree with the fused one bit for bit
+        sel2 = torch.empty_like(sel)
+        w2 = torch.empty_like(w)
+        m.select_topk(logits, probs, cfg["k"], sel2, w2)
+        torch.cuda.synchronize()
+        assert torch.equal(sel, sel2) and torch.equal(w, w2)
+    ws = m.alloc_workspace(c, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    offsets = torch.empty(c.n_heavy + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(na, dtype=torch.int32, device=dev)
+    row_of = torch.empty(na, dtype=torch.int32, device=dev)
+    tok_ptr = torch.empty(T + 1, dtype=torch.int32, device=dev) if r == "expert_choice" else None
+    tok_assign = torch.empty(na, dtype=torch.int32, device=dev) if r == "expert_choice" else None
+    x_perm = torch.empty(na, d, dtype=inp["x"].dtype, device=dev)
+    m.dispatch(c, sel, inp["x"], x_perm, offsets, perm, row_of, tok_ptr, tok_assign, status, ws)
+    torch.cuda.synchronize()
+    out = {"logits": logits.cpu().numpy(), "probs": probs.cpu().numpy(),
+           "sel": sel.cpu().numpy(), "w": w.cpu().numpy()}
+    gsel = H.selection_of(cfg, out)
+    a_tok, a_exp, _ = oracle.assignments_from_selection(cfg, gsel)
+    o_off, o_perm, o_row, o_tptr, o_tass = oracle.dispatch(a_tok, a_exp, cfg["E_heavy"], T)
+    n_rows = int(o_off[-1])
+    np.testing.assert_array_equal(offsets.cpu().numpy(), o_off)
+    np.testing.assert_array_equal(perm.cpu().numpy()[:n_rows], o_perm)
+    np.testing.assert_array_equal(row_of.cpu().numpy(), o_row)
+    if r == "expert_choice":
+        np.testing.assert_array_equal(tok_ptr.cpu().numpy(), o_tptr)
+        np.testing.assert_array_equal(tok_assign.cpu().numpy(), o_tass)
+    assert torch.equal(x_perm[:n_rows], inp["x"][perm[:n_rows].long()])
+
+    y_perm = torch.empty(na, d, device=dev)
+    y_sh = torch.empty(T, d, device=dev) if cfg["n_shared"] else None
+    m.grouped_mlp(c, x_perm, offsets, inp["W1"], inp["W2"], inp["x"], inp["Ws1"], inp["Ws2"],
+                  y_perm, y_sh, status, ws)
+    torch.cuda.synchronize()
+    yp = y_perm.cpu().numpy()[:n_rows]
+    ref_rows = np.empty_like(yp, dtype=np.float64)
+    for e in range(cfg["E_heavy"]):
+        lo, hi = o_off[e], o_off[e + 1]
+        if hi > lo:
+            ref_rows[lo:hi] = oracle.heavy_expert(cfg["act"], hin["x"][o_perm[lo:hi]],
+                                                  hin["W1"][e], hin["W2"][e], cfg["h"])
+    assert H.normwise(yp, ref_rows) <= H.Y_TOL[cfg["dtype"]]
+    if y_sh is not None:
+        ref_sh = oracle.mlp_gelu(hin["x"], hin["Ws1"], hin["Ws2"])
+        assert H.normwise(y_sh.cpu().numpy(), ref_sh) <= H.Y_TOL[cfg["dtype"]]
+
+    y = torch.empty_like(inp["x"])
+    m.combine(c, y_perm, y_sh, sel, w, row_of, tok_ptr, tok_assign, inp["x"],
+              inp["const_vecs"], inp["x"], y, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    y_ref = H.oracle_layer(cfg, hin, gsel)
+    assert H.normwise(gen.to_numpy_f32(y), y_ref) <= H.Y_TOL[cfg["dtype"]]
+
+
+# ---------------------------------------------------------------- edge cases
+EDGE = [
+    ("empty", "ditmoe_xl", dict(T=0, d=256, h=512, h_shared=256)),
+    ("one_token", "ditmoe_xl", dict(T=1, d=256, h=512, h_shared=256)),
+    ("single_expert", "ditmoe_xl", dict(T=300, d=128, E=1, k=1, h=256, n_shared=0)),
+    ("k_equals_E", "ditmoe_xl", dict(T=130, d=128, E=4, k=4, h=256, n_shared=0)),
+    ("E_128", "ditmoe_xl", dict(T=257, d=128, E=128, k=8, h=128, n_shared=0)),
+    ("all_zero_compute", "mmoe", dict(T=200, d=128, h=256, h_shared=128, zero_compute_logit_bias=60.0)),
+    ("ec_full_capacity", "ecdit", dict(T=64, group_size=16, d=128, E=4, h=256, capacity=16)),
+    ("ec_whole_batch", "ecdit", dict(T=2048, group_size=2048, d=128, E=8, h=256, capacity=512)),
+    ("des_beta_one", "des_vote", dict(d=128, h=128, M_core=64)),
+    ("odd_N_swiglu_routed", "des_vote", dict(T=37, d=128, E=16, k=4, h=128, M_core=8)),
+    ("tiny_fp32_k1", "tiny_fp32", dict(k=1)),
+]
+
+
+@pytest.mark.parametrize("label,name,over", EDGE, ids=[e[0] for e in EDGE])
+def test_edge_cases(label, name, over):
+    cfg = gen.workload(name, **over)
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    assert out["status"] == 0
+    if cfg["T"] == 0:
+        return
+    hin = H.host(inp)
+    _check_router(cfg, hin, out)
+    sel = _check_selection(cfg, out)
+    y_ref = H.oracle_layer(cfg, hin, sel)
+    assert H.normwise(out["y"], y_ref) <= H.Y_TOL[cfg["dtype"]]
+    if label == "all_zero_compute":
+        assert int(out["offsets"][-1]) == 0  # no heavy rows: no GEMM tiles at all
+
+
+def test_deterministic_bytes():
+    cfg = gen.workload("mmoe", T=600, d=256, h=512, h_shared=256)
+    inp = gen.make_inputs(cfg, "cuda")
+    a = H.run_layer(cfg, inp)
+    b = H.run_layer(cfg, inp)
+    assert np.array_equal(a["y"].view(np.uint32), b["y"].view(np.uint32))
+
+
+def test_bad_indices_are_flagged_not_faulted():
+    # Host-side fault injection: corrupt expert ids in a selection; the
+    # dispatch kernel's bounds checks flag them and drop those assignments.
+    m = H.moe()
+    cfg = gen.workload("ditmoe_xl", T=64, d=128, h=256, n_shared=0)
+    c = m.make_config(cfg)
+    na = m.num_assignments(c)
+    g = torch.Generator(device="cpu").manual_seed(5)
+    sel = torch.randint(0, cfg["E"], (na,), generator=g, dtype=torch.int32)
+    sel[3] = 99
+    sel[10] = -1
+    sel = sel.cuda()
+    x = torch.randn(cfg["T"], cfg["d"], device="cuda").to(torch.bfloat16)
+    ws = m.alloc_workspace(c)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(c.n_heavy + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(na, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(na, dtype=torch.int32, device="cuda")
+    m.dispatch(c, sel, x, None, offsets, perm, row_of, None, None, status, ws)
+    torch.cuda.synchronize()
+    assert int(status.item()) & m.DEV_BAD_EXPERT
+    ro = row_of.cpu().numpy()
+    assert ro[3] == -1 and ro[10] == -1
+    assert int(offsets[-1].item()) == na - 2
