@@ -33,6 +33,21 @@ METRIC = "MoE-layer tokens/s and TFLOP/s (or HBM GB/s) vs B200 roofline, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the grouped-MLP
+# launches of one layer pass, from one ncu capture (profiles/), valid only while
+# the GEMM kernel source is byte-identical to the one profiled.
+NCU_TRAFFIC = {
+    "ditmoe_xl": {"bytes": (163.87 + 252.31 + 500.84 + 97.23) * 1e6,
+                  "gemm_source_sha256_16": "b9d44b6780bae36a"},
+}
+
+
+def gemm_source_hash():
+    import hashlib
+    path = os.path.join(ROOT, "mixture_experts_layer_33_b200", "csrc", "gemm_sm100.cu")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
 
 # ------------------------------------------------------------- bookkeeping
 def describe(cfg):
@@ -92,54 +107,97 @@ def aggregate_throughput(units_per_rank, world, max_seconds):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """SM clock and clock-event (throttle) reasons sampled every few ms by
+    NVML from a background thread while the timed region runs; falls back
+    to nvidia-smi polling if NVML is unavailable."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
 
-    def __init__(self, device_index):
-        self.idx = device_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+    def __init__(self, torch_device, period_s=0.002):
+        self.dev = torch_device
+        self.period = period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = None
+        self._thread = None
+        self._smi = None
+
+    def _handle(self, pynvml):
+        import torch
+        try:
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
 
     def start(self):
+        import threading
         try:
-            self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=self.out, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            h = self._handle(pynvml)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            self._start_smi()
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                    bits = int(get_reasons(h))
+                    for n, b in self.REASON_BITS.items():
+                        if bits & b:
+                            self.reasons.add(n)
+                except Exception:
+                    pass
+                time.sleep(self.period)
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+
+    def _start_smi(self):
+        self.path = os.path.join("/tmp", f"moe_bench_clocks_{os.getpid()}.csv")
+        try:
+            self._out = open(self.path, "w")
+            self._smi = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=clocks.sm,clocks.max.sm,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self._out, stderr=subprocess.DEVNULL)
         except OSError:
-            self.proc = None
+            self._smi = None
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                cols = [c.strip() for c in line.split(",")]
-                if len(cols) < 9:
-                    continue
-                try:
-                    sm.append(float(cols[1]))
-                    smax = float(cols[2])
-                except ValueError:
-                    continue
-                for n, v in zip(names, cols[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(n)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        elif self._smi is not None:
+            self._smi.terminate()
+            self._smi.wait(timeout=5)
+            self._out.close()
+            names = ["hw_slowdown", "sw_thermal_slowdown", "hw_thermal_slowdown", "sw_power_cap"]
+            with open(self.path) as f:
+                for line in f:
+                    cols = [c.strip() for c in line.split(",")]
+                    try:
+                        self.samples.append(float(cols[0]))
+                        self.max_mhz = float(cols[1])
+                    except (ValueError, IndexError):
+                        continue
+                    for n, v in zip(names, cols[2:6]):
+                        if v.lower() == "active":
+                            self.reasons.add(n)
+            os.unlink(self.path)
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
 
 
 # ----------------------------------------------------------- GPU benchmark
@@ -246,9 +304,8 @@ def gpu_bench(args):
     flops = mlp_flops(cfg, n_rows)
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(dev)
     sampler.start()
-    time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -298,20 +355,22 @@ def gpu_bench(args):
     h2d = act_bytes + (cfg["T"] * cfg["E"] * 4 if zp_h is not None else 0)
 
     peaks, peak_src = load_peaks()
+    tr = NCU_TRAFFIC.get(cfg["name"])
+    traffic = tr["bytes"] if tr and tr["gemm_source_sha256_16"] == gemm_source_hash() else None
     gm_ms = stage_ms["grouped_mlp"] / args.steps
     if cfg["routing"] == "des_vote":
         bytes_ = weight_bytes_used(cfg, used)
         achieved = bytes_ / (gm_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": "grouped_mlp (GEMM1 + GEMM2 launches)",
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "algorithmic_per_launch": bytes_, "peak_source": peak_src}
     else:
         achieved = flops / (gm_ms / 1e3) / 1e12
         pk = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "kernel": "grouped_mlp (GEMM1 + GEMM2 launches)",
                 "achieved": round(achieved, 1), "peak": pk, "unit": "TFLOP/s",
-                "frac": round(achieved / pk, 4), "traffic": None,
+                "frac": round(achieved / pk, 4), "traffic": traffic,
                 "algorithmic_per_launch": flops, "peak_source": peak_src + " (burst)"}
 
     line = {
@@ -435,7 +494,7 @@ def reference_bench(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
