@@ -216,6 +216,36 @@ MOE_API int moe_dispatch(const moe_config *cfg, const int32_t *sel, const void *
                  int32_t *tok_ptr, int32_t *tok_assign, int32_t *dev_status,
                  void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Bytes of library-owned device scratch behind moe_dispatch_noalloc. */
+#define MOE_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+
+/*
+ * moe_dispatch without a workspace: the same dispatch, with the same
+ * arguments, layouts and outputs as moe_dispatch minus ws / ws_bytes.
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory (for example a host framework that
+ * owns all device memory and forbids allocation outside its own pool, or a
+ * latency-critical path that cannot afford cudaMalloc's implicit
+ * synchronisation) and so cannot hand over a workspace.
+ *   - It allocates nothing. Its scratch (the per-block expert histograms)
+ *     is a fixed file-scope __device__ array of MOE_NOALLOC_SCRATCH_BYTES
+ *     that every GPU loading the library holds until the process exits.
+ *   - Limit: ceil(n_assign / 1024) * n_heavy * 4 bytes must fit in
+ *     MOE_NOALLOC_SCRATCH_BYTES; larger configurations return
+ *     MOE_ERR_UNSUPPORTED before anything is launched (use moe_dispatch).
+ *   - The first call on a device, made with that device current, looks up
+ *     the array's device address once (cudaGetSymbolAddress) and caches
+ *     it; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (the kernels overwrite every entry they read, so nothing needs
+ *     clearing). Calls that overlap on the GPU race on it: serialise them.
+ */
+MOE_API int moe_dispatch_noalloc(const moe_config *cfg, const int32_t *sel,
+                                 const void *x, void *x_perm, int32_t *offsets,
+                                 int32_t *perm, int32_t *row_of,
+                                 int32_t *tok_ptr, int32_t *tok_assign,
+                                 int32_t *dev_status, moe_stream_t stream);
+
 /*
  * Grouped expert MLP over the dispatched rows, plus the shared expert(s).
  * MMOE page, "MoE++ expert layer" (heavy experts are standard MLPs) and

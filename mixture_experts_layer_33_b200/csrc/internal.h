@@ -54,6 +54,9 @@ struct DispatchArgs {
 };
 size_t dispatch_workspace_bytes(int64_t n_assign, int n_heavy);
 int launch_dispatch(const DispatchArgs &a, void *ws, cudaStream_t stream);
+// dispatch_noalloc.cu: the dispatch with library-owned scratch.
+bool dispatch_fits_noalloc_scratch(int64_t n_assign, int n_heavy);
+int launch_dispatch_noalloc(const DispatchArgs &a, cudaStream_t stream);
 int launch_gather_rows(const void *x, void *x_perm, const int32_t *perm,
                        const int32_t *offsets, int n_heavy, int64_t max_rows,
                        int d, int elem_bytes, cudaStream_t stream);

@@ -374,6 +374,24 @@ int moe_dispatch(const moe_config *cfg, const int32_t *sel, const void *x, void 
                             elem_bytes(c.dtype), stream);
 }
 
+int moe_dispatch_noalloc(const moe_config *cfg, const int32_t *sel, const void *x, void *x_perm,
+                         int32_t *offsets, int32_t *perm, int32_t *row_of, int32_t *tok_ptr,
+                         int32_t *tok_assign, int32_t *dev_status, moe_stream_t stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config &c = *cfg;
+  if (!offsets) return MOE_ERR_INVALID_ARG;
+  if (n_assign_of(c) > 0 && (!sel || !perm || !row_of)) return MOE_ERR_INVALID_ARG;
+  if (x_perm && (!x || !aligned16(x) || !aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
+  if (c.routing == MOE_EXPERT_CHOICE && (!tok_ptr != !tok_assign)) return MOE_ERR_INVALID_ARG;
+  if (!dispatch_fits_noalloc_scratch(n_assign_of(c), c.n_heavy)) return MOE_ERR_UNSUPPORTED;
+  DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
+  st = launch_dispatch_noalloc(da, stream);
+  if (st != MOE_OK || !x_perm || c.n_heavy == 0) return st;
+  return launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, n_assign_of(c), c.d,
+                            elem_bytes(c.dtype), stream);
+}
+
 int moe_grouped_mlp(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
                     const void *W1, const void *W2, const void *x, const void *Ws1,
                     const void *Ws2, float *y_perm, float *y_shared, int32_t *dev_status,

@@ -30,7 +30,9 @@ ENTRY_POINTS = (
     "moe_workspace_size", "moe_router", "moe_select_topk",
     "moe_select_expert_choice", "moe_core_set_vote", "moe_dispatch",
     "moe_grouped_mlp", "moe_combine", "moe_forward", "moe_forward_host",
+    "moe_dispatch_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 256 * 1024  # MOE_NOALLOC_SCRATCH_BYTES
 
 
 class MoeConfig(ctypes.Structure):
@@ -63,6 +65,7 @@ _SIGS = {
     "moe_select_expert_choice": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_core_set_vote": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_dispatch": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_dispatch_noalloc": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_grouped_mlp": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                _vp]),
     "moe_combine": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -202,6 +205,29 @@ def dispatch(c: MoeConfig, sel, x, x_perm, offsets, perm, row_of, tok_ptr, tok_a
                             _dev_ptr(offsets), _dev_ptr(perm), _dev_ptr(row_of),
                             _dev_ptr(tok_ptr), _dev_ptr(tok_assign), _dev_ptr(dev_status),
                             _dev_ptr(ws), ws.numel(), _stream(stream)), "moe_dispatch")
+
+
+def dispatch_noalloc(c: MoeConfig, sel, x, x_perm, offsets, perm, row_of, tok_ptr, tok_assign,
+                     dev_status, stream=None):
+    """moe_dispatch for callers that cannot allocate device memory.
+
+    Same arguments and outputs as ``dispatch`` minus the workspace: the
+    library keeps the histogram scratch in a fixed device array of
+    NOALLOC_SCRATCH_BYTES per GPU. Configurations whose scratch would not
+    fit (ceil(n_assign/1024) * n_heavy * 4 bytes) are rejected. The first
+    call on a device sets up the array's address (make it before any stream
+    capture); calls that overlap on the GPU share the array and race.
+    """
+    code = LIB.moe_dispatch_noalloc(ctypes.byref(c), _dev_ptr(sel), _dev_ptr(x),
+                                    _dev_ptr(x_perm), _dev_ptr(offsets), _dev_ptr(perm),
+                                    _dev_ptr(row_of), _dev_ptr(tok_ptr), _dev_ptr(tok_assign),
+                                    _dev_ptr(dev_status), _stream(stream))
+    if code == 2:
+        raise RuntimeError(
+            "moe_dispatch_noalloc failed: the configuration's dispatch scratch "
+            f"(ceil(n_assign/1024) * n_heavy * 4 bytes) exceeds the {NOALLOC_SCRATCH_BYTES}-byte "
+            "library-owned array; use dispatch() with a workspace")
+    _check(code, "moe_dispatch_noalloc")
 
 
 def grouped_mlp(c: MoeConfig, x_perm, offsets, W1, W2, x, Ws1, Ws2, y_perm, y_shared,
