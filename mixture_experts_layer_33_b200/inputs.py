@@ -63,7 +63,7 @@ WORKLOADS = {
 # those three experts so that roughly that share of the routed slots lands
 # on them. The value was calibrated with the oracle's routing by
 # tests/golden/calibrate_mmoe_skew.py.
-MMOE_SKEW_BIAS = 1.0
+MMOE_SKEW_BIAS = 0.791
 WORKLOADS["mmoe_skewed"] = dict(WORKLOADS["mmoe"], zero_compute_logit_bias=MMOE_SKEW_BIAS)
 
 
