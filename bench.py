@@ -4,10 +4,11 @@
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
 
 A step is one pass of the whole layer (router + softmax + selection ->
-dispatch -> grouped expert MLP -> combine) over one batch of synthetic input,
-issued as the library's staged C-ABI calls on one stream with a CUDA event
-between stages; the same launches moe_forward makes. L2 is flushed (a
-256 MiB write) before every timed step, outside the events. ``value`` is
+dispatch -> grouped expert MLP -> combine) over one batch of synthetic input
+through moe_forward, replayed as a CUDA graph; a second timed loop issues
+the same layer as the staged C-ABI calls with a CUDA event between stages
+for the per-stage split and the grouped MLP's own duration. L2 is flushed
+(a 256 MiB write) before every timed step, outside the events. ``value`` is
 tokens/s over the K timed steps (inputs resident in HBM); ``e2e`` repeats
 the measurement through moe_forward_host with the activations in pinned
 host memory and the copies inside the timed region. Multi-GPU runs are
@@ -231,11 +232,30 @@ class StagedLayer:
         self.status = torch.zeros(1, dtype=torch.int32, **f)
         self.stages = ["router+select", "dispatch", "grouped_mlp", "combine"]
         self.launches = {"router+select": 1 + (cfg["routing"] != "token_topk"),
-                         "dispatch": 4 + (1 if ec else 0),
-                         "grouped_mlp": 2,
+                         "dispatch": (1 if na <= 1024 else 3) + (1 if self.c.n_heavy else 0)
+                         + (1 if ec else 0),
+                         "grouped_mlp": self._mlp_launches(cfg),
                          "combine": 1}
-        if cfg["n_shared"] and (cfg["dtype"] != "bf16" or cfg["act"] != "gelu"):
-            self.launches["grouped_mlp"] = 3 if cfg["dtype"] == "bf16" else 4
+
+    @staticmethod
+    def _mlp_launches(cfg):
+        routed = 1 if cfg["E_heavy"] else 0
+        shared = 1 if cfg["n_shared"] else 0
+        if cfg["dtype"] != "bf16":
+            return 2 * (routed + shared)
+        if cfg["T"] <= 128:  # weight-streaming kernel: one launch per problem
+            return routed + shared
+        if routed and shared:
+            return 2 if cfg["act"] == "gelu" else 3
+        return 2 * (routed + shared)
+
+    def run_forward(self):
+        """The whole layer through the single entry point moe_forward."""
+        i = self.inp
+        self.m.forward(self.c, i["x"], i["W_r"], i["W1"], i["W2"], self.y, self.ws,
+                       residual=i["x"], z_prev=i["z_prev"], bias=i["logit_bias"],
+                       Ws1=i["Ws1"], Ws2=i["Ws2"], const_vecs=i["const_vecs"],
+                       dev_status=self.status)
 
     def run(self, events=None):
         m, cfg, i = self.m, self.cfg, self.inp
@@ -303,7 +323,27 @@ def gpu_bench(args):
     used = sum(1 for a, b in zip(offs[:-1], offs[1:]) if b > a)
     flops = mlp_flops(cfg, n_rows)
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # The layer (moe_forward) as one CUDA graph; eager if capture is refused.
+    for _ in range(2):
+        layer.run_forward()
+    torch.cuda.synchronize()
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                layer.run_forward()
+            for _ in range(3):
+                flush.fill_(1)
+                graph.replay()
+            torch.cuda.synchronize()
+        except Exception as exc:  # noqa: BLE001
+            graph = None
+            print(f"graph capture unavailable: {exc}", file=sys.stderr)
+
+    # Timed region 1 (value): K layer passes, L2 flushed before each.
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
     sampler = ClockSampler(dev)
     sampler.start()
     if world > 1:
@@ -311,21 +351,33 @@ def gpu_bench(args):
     torch.cuda.synchronize()
     for s in range(args.steps):
         flush.fill_(s & 255)
-        layer.run(ev[s])
+        ev[s][0].record()
+        if graph is not None:
+            graph.replay()
+        else:
+            layer.run_forward()
+        ev[s][1].record()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    stage_ms = {n: 0.0 for n in layer.stages}
-    total_ms = 0.0
-    for s in range(args.steps):
-        for j, n in enumerate(layer.stages):
-            t = ev[s][j].elapsed_time(ev[s][j + 1])
-            stage_ms[n] += t
-            total_ms += t
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
     max_s = reduce_max_over_ranks(total_ms / 1e3, dist if world > 1 else None)
     ms_per_step = max_s * 1e3 / args.steps
     value = aggregate_throughput(cfg["T"] * args.steps, world, max_s)
+
+    # Timed region 2: the same passes as staged calls with an event between
+    # stages, for the per-stage split and the dominant kernel's duration.
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        flush.fill_(s & 255)
+        layer.run(sev[s])
+    torch.cuda.synchronize()
+    stage_ms = {n: 0.0 for n in layer.stages}
+    for s in range(args.steps):
+        for j, n in enumerate(layer.stages):
+            stage_ms[n] += sev[s][j].elapsed_time(sev[s][j + 1])
 
     # End to end through moe_forward_host: pinned host activations, copies timed.
     x_h = inp["x"].cpu().pin_memory()
@@ -357,7 +409,7 @@ def gpu_bench(args):
     peaks, peak_src = load_peaks()
     tr = NCU_TRAFFIC.get(cfg["name"])
     traffic = tr["bytes"] if tr and tr["gemm_source_sha256_16"] == gemm_source_hash() else None
-    gm_ms = stage_ms["grouped_mlp"] / args.steps
+    gm_ms = stage_ms["grouped_mlp"] / args.steps  # grouped-MLP launches, from timed region 2
     if cfg["routing"] == "des_vote":
         bytes_ = weight_bytes_used(cfg, used)
         achieved = bytes_ / (gm_ms / 1e3) / 1e9
@@ -382,6 +434,8 @@ def gpu_bench(args):
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "l2": "flushed by a 256 MiB write before every timed step"},
         "layer_tflops": round(flops / (ms_per_step / 1e3) / 1e12, 1),
+        "layer_weight_gbs": round(weight_bytes_used(cfg, used) / (ms_per_step / 1e3) / 1e9, 1),
+        "cuda_graph": graph is not None,
         "stage_ms": {k: round(v / args.steps, 4) for k, v in stage_ms.items()},
         "heavy_rows": n_rows, "experts_used": used,
         "roofline": roof,
@@ -500,6 +554,7 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

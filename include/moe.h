@@ -288,6 +288,19 @@ MOE_API int moe_combine(const moe_config *cfg, const float *y_perm,
                 const void *const_vecs, const void *residual, void *y,
                 int32_t *dev_status, moe_stream_t stream);
 
+/*
+ * The elementwise activation the heavy experts apply, on its own:
+ * act == MOE_GELU_ERF: y = GELU(x) = x * Phi(x), the exact (erf) form;
+ * act == MOE_SWIGLU:   y = SiLU(x) = x / (1 + exp(-x)), SwiGLU's gate.
+ * MMOE page, "MoE++ expert layer" (heavy experts are standard MLPs). The
+ * same device functions run in the GEMM epilogues; erf is evaluated by
+ * Abramowitz & Stegun 7.1.26 (absolute error <= 1.5e-7; below 6e-7 as
+ * evaluated in fp32, so GELU(x) is within 3e-7 |x| of the exact value).
+ *   x, y [n] fp32 device (y may alias x).
+ */
+MOE_API int moe_activation(const float *x, float *y, int64_t n, int act,
+                           moe_stream_t stream);
+
 /* Optional outputs of moe_forward (each pointer nullable; device memory). */
 typedef struct moe_forward_aux {
   float *logits;     /* [T, E] fp32 */

@@ -42,8 +42,14 @@ __device__ __forceinline__ bool decode(const DispatchArgs &a, int64_t i, int &to
   return true;
 }
 
+__device__ __forceinline__ void clear_words(const DispatchArgs &a) {
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < a.n_zero_words; i += blockDim.x) a.zero_words[i] = 0;
+}
+
 __global__ void __launch_bounds__(kThreads) dispatch_count_kernel(DispatchArgs a, int32_t *partial) {
   __shared__ int hist[MOE_MAX_EXPERTS];
+  clear_words(a);
   for (int e = threadIdx.x; e < a.n_heavy; e += kThreads) hist[e] = 0;
   __syncthreads();
   const int64_t base = (int64_t)blockIdx.x * kChunk;
@@ -79,9 +85,11 @@ __global__ void __launch_bounds__(kThreads) dispatch_scan_kernel(DispatchArgs a,
   if (e == 0) a.offsets[a.n_heavy] = all;
 }
 
-__global__ void __launch_bounds__(kThreads) dispatch_scatter_kernel(DispatchArgs a, const int32_t *base_rows) {
-  __shared__ int run[MOE_MAX_EXPERTS];
-  __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
+// Stable scatter of one chunk of kChunk assignments starting at `base`;
+// base_rows[e] is the first row of this chunk's expert-e rows.
+__device__ __forceinline__ void scatter_chunk(const DispatchArgs &a, int64_t base,
+                                              const int32_t *base_rows, int *run,
+                                              int (*wcnt)[MOE_MAX_EXPERTS]) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < a.n_heavy; e += kThreads) {
     run[e] = 0;
@@ -89,7 +97,6 @@ __global__ void __launch_bounds__(kThreads) dispatch_scatter_kernel(DispatchArgs
     for (int w = 0; w < kWarps; ++w) wcnt[w][e] = 0;
   }
   __syncthreads();
-  const int64_t base = (int64_t)blockIdx.x * kChunk;
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int r = 0; r < kPerThread; ++r) {
     const int64_t i = base + r * kThreads + tid;
@@ -103,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) dispatch_scatter_kernel(DispatchArgs
     if (key >= 0) {
       int before = run[key] + rank_w;
       for (int w = 0; w < warp; ++w) before += wcnt[w][key];
-      const int row = base_rows[(size_t)blockIdx.x * a.n_heavy + key] + before;
+      const int row = base_rows[key] + before;
       a.perm[row] = tok;
       a.row_of[i] = row;
     } else if (i < a.n_assign) {
@@ -118,6 +125,41 @@ __global__ void __launch_bounds__(kThreads) dispatch_scatter_kernel(DispatchArgs
     }
     __syncthreads();
   }
+}
+
+__global__ void __launch_bounds__(kThreads) dispatch_scatter_kernel(DispatchArgs a, const int32_t *base_rows) {
+  __shared__ int run[MOE_MAX_EXPERTS];
+  __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
+  scatter_chunk(a, (int64_t)blockIdx.x * kChunk, base_rows + (size_t)blockIdx.x * a.n_heavy, run,
+                wcnt);
+}
+
+// All assignments fit one chunk: histogram, scan and scatter in one block.
+__global__ void __launch_bounds__(kThreads) dispatch_single_block_kernel(DispatchArgs a) {
+  __shared__ int hist[MOE_MAX_EXPERTS];
+  __shared__ int32_t offs[MOE_MAX_EXPERTS];
+  __shared__ int scratch[33];
+  __shared__ int run[MOE_MAX_EXPERTS];
+  __shared__ int wcnt[kWarps][MOE_MAX_EXPERTS];
+  clear_words(a);
+  for (int e = threadIdx.x; e < a.n_heavy; e += kThreads) hist[e] = 0;
+  __syncthreads();
+  for (int r = 0; r < kPerThread; ++r) {
+    int64_t i = r * kThreads + threadIdx.x;
+    int tok, exp;
+    if (i < a.n_assign && decode(a, i, tok, exp) && exp < a.n_heavy) atomicAdd(&hist[exp], 1);
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  int all;
+  int off = block_exclusive_scan(e < a.n_heavy ? hist[e] : 0, scratch, &all);
+  if (e < a.n_heavy) {
+    offs[e] = off;
+    a.offsets[e] = off;
+  }
+  if (e == 0) a.offsets[a.n_heavy] = all;
+  __syncthreads();
+  scatter_chunk(a, 0, offs, run, wcnt);
 }
 
 // Expert choice: each token's assignments in slot order, one block per
@@ -190,6 +232,10 @@ int launch_dispatch(const DispatchArgs &a, void *ws, cudaStream_t stream) {
   const int nb = (int)((a.n_assign + kChunk - 1) / kChunk);
   if (nb == 0) {
     MOE_CUDA_TRY(cudaMemsetAsync(a.offsets, 0, (a.n_heavy + 1) * sizeof(int32_t), stream));
+    if (a.n_zero_words > 0)
+      MOE_CUDA_TRY(cudaMemsetAsync(a.zero_words, 0, a.n_zero_words * sizeof(int32_t), stream));
+  } else if (nb == 1) {
+    dispatch_single_block_kernel<<<1, kThreads, 0, stream>>>(a);
   } else {
     dispatch_count_kernel<<<nb, kThreads, 0, stream>>>(a, partial);
     dispatch_scan_kernel<<<1, kThreads, 0, stream>>>(a, partial, nb);

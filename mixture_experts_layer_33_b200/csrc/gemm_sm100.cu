@@ -29,15 +29,18 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
 
+using namespace tc;
+
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle atom row
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                    // two per TMEM lane quadrant
+constexpr int kThreads = 64 + 32 * kEpiWarps;   // producer warp, MMA warp, epilogue warps
 constexpr int kMaxEntries = 2 * MOE_MAX_EXPERTS + 2;
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s per wait
 
 struct ProbDev {
   const int32_t *offsets;
@@ -47,6 +50,7 @@ struct ProbDev {
   int N, K;
   void *out;
   int64_t ld_out;
+  int vec32;  // rows of `out` start on 32-byte boundaries: 256-bit stores
 };
 struct ParamsDev {
   int n_probs;
@@ -64,118 +68,6 @@ struct Sched {
   int row_end[kMaxEntries];
 };
 
-// ---------------------------------------------------------------- PTX
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait. Returns false if the kernel is aborting (another role gave
-// up) or this wait expired (then it raises the abort itself).
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       int32_t *status, bool watch_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t spin = 1;; ++spin) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((spin & 63u) == 0) {
-      if (watch_abort && *abort_flag) return false;
-      if (global_timer_ns() - t0 > kTimeoutNs) {
-        *abort_flag = 1;
-        set_status(status, MOE_DEV_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-// D[tmem] (+)= A[smem] . B[smem]^T, M=128, N from the instruction descriptor, K=16.
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle,
-// 8-row core groups 1024 bytes apart (SBO), descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);        // start address
-  d |= (uint64_t)1u << 16;                        // leading byte offset (unused for SW128 K-major)
-  d |= (uint64_t)(1024u >> 4) << 32;              // stride byte offset
-  d |= (uint64_t)1u << 46;                        // version (sm_100)
-  d |= (uint64_t)2u << 61;                        // layout: SWIZZLE_128B
-  return d;
-}
-
-// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M=128, N=n.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int n) {
-  return (1u << 4)                       // D format f32
-         | (1u << 7)                     // A format bf16
-         | (1u << 10)                    // B format bf16
-         | ((uint32_t)(n >> 3) << 17)    // N / 8
-         | ((uint32_t)(BM >> 4) << 24);  // M / 16
-}
-
 __device__ __forceinline__ int find_entry(const Sched &s, int t) {
   int lo = 0, hi = s.n_entries - 1;
   while (lo < hi) {
@@ -183,6 +75,59 @@ __device__ __forceinline__ int find_entry(const Sched &s, int t) {
     if (s.tile_start[mid] <= t) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+
+__device__ __forceinline__ void st_global_v8(void *p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// 32 consecutive output columns of one row: whole 32-byte sectors per
+// store when rows are 32-byte aligned, 16-byte stores otherwise, scalar
+// stores at a ragged right edge.
+template <bool OUT_F32>
+__device__ __forceinline__ void store_row32(const ProbDev &pr, int row, int col, const float (&v)[32]) {
+  if (OUT_F32) {
+    float *o = static_cast<float *>(pr.out) + (int64_t)row * pr.ld_out + col;
+    if (col + 32 <= pr.N) {
+      if (pr.vec32) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint32_t w[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) w[j] = __float_as_uint(v[i + j]);
+          st_global_v8(o + i, w);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4 *>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    } else {
+      for (int i = 0; i < 32 && col + i < pr.N; ++i) o[i] = v[i];
+    }
+  } else {
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(pr.out) + (int64_t)row * pr.ld_out + col;
+    if (col + 32 <= pr.N) {
+      uint32_t w[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        w[j] = *reinterpret_cast<uint32_t *>(&h2);
+      }
+      if (pr.vec32) {
+        st_global_v8(o, *reinterpret_cast<const uint32_t(*)[8]>(&w[0]));
+        st_global_v8(o + 16, *reinterpret_cast<const uint32_t(*)[8]>(&w[8]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          *reinterpret_cast<uint4 *>(o + 8 * i) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+      }
+    } else {
+      for (int i = 0; i < 32 && col + i < pr.N; ++i) o[i] = __float2bfloat16_rn(v[i]);
+    }
+  }
 }
 
 template <int BN, int ACT, bool OUT_F32, int STAGES>
@@ -195,7 +140,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
-  constexpr uint32_t IDESC = idesc_bf16_f32(BN);
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
@@ -222,7 +167,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull0 + 8 * a, 1);
-      mbar_init(tempty0 + 8 * a, 4);
+      mbar_init(tempty0 + 8 * a, kEpiWarps);
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -344,8 +289,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
     mbar_wait(drain, 0, &abort_flag, p.status, false);
   } else if (warp >= 2) {
     // ---------------- epilogue
-    const int quad = warp & 3;
+    const int quad = warp & 3;                  // TMEM lanes this warp may read
     const int lrow = quad * 32 + lane;
+    const int c_lo = ((warp - 2) / 4) * (BNO / 2);  // this warp's half of the columns
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
@@ -364,7 +310,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
 #pragma unroll 1
-      for (int c = 0; c < BNO; c += 32) {
+      for (int c = c_lo; c < c_lo + BNO / 2; c += 32) {
         float v[32];
         tmem_ld32(taddr + c, v);
         if (ACT == kActSwiglu) {
@@ -376,33 +322,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
         }
-        if (valid) {
-          const int col = col0 + c;
-          if (OUT_F32) {
-            float *o = static_cast<float *>(pr.out) + (int64_t)row * pr.ld_out + col;
-            if (col + 32 <= pr.N) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(o + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-            } else {
-              for (int i = 0; i < 32 && col + i < pr.N; ++i) o[i] = v[i];
-            }
-          } else {
-            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(pr.out) + (int64_t)row * pr.ld_out + col;
-            if (col + 32 <= pr.N) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 8) {
-                uint4 u4;
-                __nv_bfloat162 *h2 = reinterpret_cast<__nv_bfloat162 *>(&u4);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) h2[j] = __floats2bfloat162_rn(v[i + 2 * j], v[i + 2 * j + 1]);
-                *reinterpret_cast<uint4 *>(o + i) = u4;
-              }
-            } else {
-              for (int i = 0; i < 32 && col + i < pr.N; ++i) o[i] = __float2bfloat16_rn(v[i]);
-            }
-          }
-        }
+        if (valid) store_row32<OUT_F32>(pr, row, col0 + c, v);
       }
       tc_fence_before();
       __syncwarp();
@@ -416,6 +336,229 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+
+// Two-SM variant: a cluster of 2 CTAs computes one 256 x BN tile with
+// tcgen05.mma.cta_group::2. Each CTA loads its own 128 rows of A and its
+// own half of the BN rows of B (for SwiGLU: gate rows in rank 0, up rows
+// in rank 1), so each SM moves 2/3 of the operand bytes the 1-SM kernel
+// does per unit of MMA work. Both CTAs' loads complete on the leader's
+// (rank 0) full barrier; the leader's single MMA thread issues the M=256
+// MMAs and releases ring slots and accumulators in both CTAs with one
+// multicast commit; both CTAs' epilogue warps read their own TMEM rows and
+// arrive on the leader's accumulator-empty barrier.
+template <int BN, int ACT, bool OUT_F32, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                         const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                         const ParamsDev p) {
+  constexpr int BMP = 2 * BM;                              // rows per pair tile
+  constexpr int BNO = (ACT == kActSwiglu) ? BN / 2 : BN;   // output columns per tile
+  constexpr uint32_t A_BYTES = BM * BK * 2;                // this CTA's rows of A
+  constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;          // this CTA's half of B
+  constexpr uint32_t STAGE_TX = 2 * (A_BYTES + B_BYTES);   // both CTAs, counted by the leader
+  constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BMP, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[2 * STAGES + 5];
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+  __shared__ Sched sched;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = (int)cluster_id_x(), npairs = (int)nclusters_x();
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~(uintptr_t)1023);
+  const uint32_t sA = smem_u32(base);
+  const uint32_t sB = sA + STAGES * A_BYTES;
+  const uint32_t full0 = smem_u32(&bars[0]);
+  const uint32_t empty0 = smem_u32(&bars[STAGES]);
+  const uint32_t tfull0 = smem_u32(&bars[2 * STAGES]);
+  const uint32_t tempty0 = smem_u32(&bars[2 * STAGES + 2]);
+  const uint32_t drain = smem_u32(&bars[2 * STAGES + 4]);
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull0 + 8 * a, 1);
+      mbar_init(tempty0 + 8 * a, 2 * kEpiWarps);  // epilogue warps of both CTAs
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  if (warp == 2) {
+    int run = 0, ne = 0;
+    for (int pi = 0; pi < p.n_probs; ++pi) {
+      const ProbDev &pr = p.pr[pi];
+      const int ntn = (pr.N + BNO - 1) / BNO;
+      for (int g0 = 0; g0 < pr.n_groups; g0 += 32) {
+        int g = g0 + lane;
+        int lo = 0, hi = 0;
+        if (g < pr.n_groups) {
+          lo = pr.offsets ? pr.offsets[g] : 0;
+          hi = pr.offsets ? pr.offsets[g + 1] : (int)pr.a_rows;
+        }
+        int tiles = (g < pr.n_groups && hi > lo) ? ((hi - lo + BMP - 1) / BMP) * ntn : 0;
+        int inc = warp_inclusive_scan(tiles);
+        if (g < pr.n_groups) {
+          const int e = ne + lane;
+          sched.tile_start[e] = run + inc - tiles;
+          sched.prob[e] = pi;
+          sched.group[e] = g;
+          sched.row0[e] = lo;
+          sched.row_end[e] = hi;
+        }
+        run += __shfl_sync(0xffffffffu, inc, 31);
+        ne += min(32, pr.n_groups - g0);
+      }
+    }
+    if (lane == 0) {
+      sched.n_entries = ne;
+      sched.total_tiles = run;
+      sched.tile_start[ne] = run;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers exist before any cross-CTA arrival
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  const int total_tiles = sched.total_tiles;
+  const uint32_t leader_full0 = mapa_shared(full0, 0);
+  const uint32_t leader_tempty0 = mapa_shared(tempty0, 0);
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0, armed = 0, armed_parity = 0;
+    bool ok = true;
+    for (int t = pair; ok && t < total_tiles; t += npairs) {
+      const int e = find_entry(sched, t);
+      const int pi = sched.prob[e];
+      const ProbDev &pr = p.pr[pi];
+      const int ntn = (pr.N + BNO - 1) / BNO;
+      const int local = t - sched.tile_start[e];
+      const int mt = local / ntn, nt = local - mt * ntn;
+      const int a_row = sched.row0[e] + mt * BMP + (int)rank * BM;
+      const int b_row = sched.group[e] * pr.b_rows_per_group + nt * BNO +
+                        (int)rank * ((ACT == kActSwiglu) ? pr.N : BN / 2);
+      const CUtensorMap *mA = pi ? &tmA1 : &tmA0;
+      const CUtensorMap *mB = pi ? &tmB1 : &tmB0;
+      const int nkb = (pr.K + BK - 1) / BK;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait_cluster(empty0 + 8 * stage, phase ^ 1u, &abort_flag, p.status)) { ok = false; break; }
+        if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, STAGE_TX);
+        const uint32_t fb = leader_full0 + 8 * stage;
+        tma_load_2d_pair(sA + stage * A_BYTES, mA, kb * BK, a_row, fb);
+        tma_load_2d_pair(sB + stage * B_BYTES, mB, kb * BK, b_row, fb);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (leader)  // the leader's full barriers count both CTAs' copies
+      for (int s = 0; s < STAGES; ++s)
+        if (armed & (1u << s))
+          mbar_wait_cluster(full0 + 8 * s, (armed_parity >> s) & 1u, &abort_flag, p.status, false);
+  } else if (warp == 1 && lane == 0) {
+    if (leader) {
+      // ---------------- MMA issuer (leader only)
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < total_tiles; t += npairs) {
+        const int e = find_entry(sched, t);
+        const int nkb = (p.pr[sched.prob[e]].K + BK - 1) / BK;
+        if (!mbar_wait_cluster(tempty0 + 8 * acc, acc_phase ^ 1u, &abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_cluster(full0 + 8 * stage, phase, &abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(sA + stage * A_BYTES);
+          const uint64_t bdesc = smem_desc_sw128(sB + stage * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_pair(d_tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), IDESC,
+                        (kb | kk) != 0 ? 1u : 0u);
+          tc_commit_pair(empty0 + 8 * stage, 0x3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(tfull0 + 8 * acc, 0x3);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      tc_commit_pair(drain, 0x3);
+    }
+    // Both CTAs: every MMA that reads this CTA's shared memory or writes its
+    // TMEM has completed once the leader's last commit lands here.
+    mbar_wait_cluster(drain, 0, &abort_flag, p.status, false);
+  } else if (warp >= 2) {
+    // ---------------- epilogue (both CTAs, own TMEM rows)
+    const int quad = warp & 3;                  // TMEM lanes this warp may read
+    const int lrow = quad * 32 + lane;
+    const int c_lo = ((warp - 2) / 4) * (BNO / 2);  // this warp's half of the columns
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < total_tiles; t += npairs) {
+      const int e = find_entry(sched, t);
+      const ProbDev &pr = p.pr[sched.prob[e]];
+      const int ntn = (pr.N + BNO - 1) / BNO;
+      const int local = t - sched.tile_start[e];
+      const int mt = local / ntn, nt = local - mt * ntn;
+      const int row = sched.row0[e] + mt * BMP + (int)rank * BM + lrow;
+      const bool valid = row < sched.row_end[e];
+      const int col0 = nt * BNO;
+      const bool ready = mbar_wait_cluster(tfull0 + 8 * acc, acc_phase, &abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+      for (int c = c_lo; c < c_lo + BNO / 2; c += 32) {
+        float v[32];
+        tmem_ld32(taddr + c, v);
+        if (ACT == kActSwiglu) {
+          float u[32];
+          tmem_ld32(taddr + BN / 2 + c, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * u[i];
+        } else if (ACT == kActGelu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+        }
+        if (valid) store_row32<OUT_F32>(pr, row, col0 + c, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(TMEM_COLS)
                  : "memory");
   }
@@ -456,6 +599,10 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, int b
   return r == CUDA_SUCCESS;
 }
 
+bool vec32_ok(const GemmProblem &q, int elem) {
+  return (reinterpret_cast<uintptr_t>(q.out) & 31u) == 0 && (q.ld_out * elem) % 32 == 0;
+}
+
 template <int BN, int ACT, bool OUT_F32>
 int run_tc(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t stream) {
   constexpr uint32_t STAGE_BYTES = (BM + BN) * BK * 2;
@@ -483,6 +630,7 @@ int run_tc(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t 
     pd.pr[i].K = q.K;
     pd.pr[i].out = q.out;
     pd.pr[i].ld_out = q.ld_out;
+    pd.pr[i].vec32 = vec32_ok(q, OUT_F32 ? 4 : 2);
     max_tiles += max_m_tiles(q, BM) * ((q.N + BNO - 1) / BNO);
   }
   if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; }
@@ -495,7 +643,68 @@ int run_tc(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t 
   return last_launch_status();
 }
 
+template <int BN, int ACT, bool OUT_F32>
+int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t stream) {
+  constexpr uint32_t STAGE_BYTES = (BM + BN / 2) * BK * 2;  // per CTA
+  constexpr int S0 = (200 * 1024) / STAGE_BYTES;
+  constexpr int STAGES = S0 > 8 ? 8 : S0;
+  constexpr int BNO = (ACT == kActSwiglu) ? BN / 2 : BN;
+  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES;
+
+  CUtensorMap maps[4];
+  memset(maps, 0, sizeof(maps));
+  ParamsDev pd;
+  memset(&pd, 0, sizeof(pd));
+  pd.n_probs = n_probs;
+  pd.status = status;
+  int64_t max_tiles = 0;
+  for (int i = 0; i < n_probs; ++i) {
+    const GemmProblem &q = probs[i];
+    if (!make_map(&maps[2 * i], q.A, q.a_rows, q.K, BM)) return MOE_ERR_CUDA;
+    if (!make_map(&maps[2 * i + 1], q.B, (int64_t)q.n_groups * q.b_rows_per_group, q.K, BN / 2))
+      return MOE_ERR_CUDA;
+    pd.pr[i].offsets = q.offsets;
+    pd.pr[i].n_groups = q.n_groups;
+    pd.pr[i].a_rows = q.a_rows;
+    pd.pr[i].b_rows_per_group = q.b_rows_per_group;
+    pd.pr[i].N = q.N;
+    pd.pr[i].K = q.K;
+    pd.pr[i].out = q.out;
+    pd.pr[i].ld_out = q.ld_out;
+    pd.pr[i].vec32 = vec32_ok(q, OUT_F32 ? 4 : 2);
+    max_tiles += max_m_tiles(q, 2 * BM) * ((q.N + BNO - 1) / BNO);
+  }
+  if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; }
+  if (max_tiles == 0) return MOE_OK;
+  auto kern = grouped_gemm_pair_kernel<BN, ACT, OUT_F32, STAGES>;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
+    return MOE_ERR_UNSUPPORTED;
+  if (max_tiles < clusters) clusters = (int)max_tiles;
+  cfg.gridDim = dim3(2 * (unsigned)clusters);
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], pd));
+  return last_launch_status();
+}
+
 }  // namespace
+
+bool make_tma_2d_bf16(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, int box_rows) {
+  return make_map(map, ptr, rows, cols, box_rows);
+}
 
 // Largest tile width whose output columns divide every problem's N.
 static int pick_bn(const GemmProblem *probs, int n_probs, int act) {
@@ -510,26 +719,50 @@ static int pick_bn(const GemmProblem *probs, int n_probs, int act) {
   return 128;
 }
 
+// The pair (2-SM) kernel pays off with full 256-wide tiles, long K (so the
+// pair's shared accumulator hand-off is amortised) and groups large enough
+// to fill 256-row tiles; measured on B200 it is slower with N=192 tiles or
+// K ~ 1152, where the single-SM kernel is used.
+static bool use_pair(const GemmProblem *probs, int n_probs, int bn) {
+  if (bn != 256) return false;
+  int64_t rows = 0, groups = 0;
+  for (int i = 0; i < n_probs; ++i) {
+    if (probs[i].K < 2048) return false;
+    rows += probs[i].a_rows;
+    groups += probs[i].offsets ? probs[i].n_groups : 1;
+  }
+  return groups > 0 && rows >= 256 * groups;
+}
+
 int launch_grouped_gemm_bf16(const GemmProblem *probs, int n_probs, int act, bool out_f32,
                              int32_t *dev_status, cudaStream_t stream) {
   if (n_probs < 1 || n_probs > 2) return MOE_ERR_INVALID_ARG;
   const int bn = pick_bn(probs, n_probs, act);
+  const bool pair = use_pair(probs, n_probs, bn);
   if (!out_f32) {
     if (act == kActGelu) {
-      if (bn == 256) return run_tc<256, kActGelu, false>(probs, n_probs, dev_status, stream);
-      if (bn == 192) return run_tc<192, kActGelu, false>(probs, n_probs, dev_status, stream);
-      return run_tc<128, kActGelu, false>(probs, n_probs, dev_status, stream);
+      if (bn == 256) return pair ? run_tc_pair<256, kActGelu, false>(probs, n_probs, dev_status, stream)
+                                 : run_tc<256, kActGelu, false>(probs, n_probs, dev_status, stream);
+      if (bn == 192) return pair ? run_tc_pair<192, kActGelu, false>(probs, n_probs, dev_status, stream)
+                                 : run_tc<192, kActGelu, false>(probs, n_probs, dev_status, stream);
+      return pair ? run_tc_pair<128, kActGelu, false>(probs, n_probs, dev_status, stream)
+                  : run_tc<128, kActGelu, false>(probs, n_probs, dev_status, stream);
     }
     if (act == kActSwiglu) {
-      if (bn == 256) return run_tc<256, kActSwiglu, false>(probs, n_probs, dev_status, stream);
-      return run_tc<128, kActSwiglu, false>(probs, n_probs, dev_status, stream);
+      if (bn == 256) return pair ? run_tc_pair<256, kActSwiglu, false>(probs, n_probs, dev_status, stream)
+                                 : run_tc<256, kActSwiglu, false>(probs, n_probs, dev_status, stream);
+      return pair ? run_tc_pair<128, kActSwiglu, false>(probs, n_probs, dev_status, stream)
+                  : run_tc<128, kActSwiglu, false>(probs, n_probs, dev_status, stream);
     }
     return MOE_ERR_UNSUPPORTED;
   }
   if (act != kActNone) return MOE_ERR_UNSUPPORTED;
-  if (bn == 256) return run_tc<256, kActNone, true>(probs, n_probs, dev_status, stream);
-  if (bn == 192) return run_tc<192, kActNone, true>(probs, n_probs, dev_status, stream);
-  return run_tc<128, kActNone, true>(probs, n_probs, dev_status, stream);
+  if (bn == 256) return pair ? run_tc_pair<256, kActNone, true>(probs, n_probs, dev_status, stream)
+                             : run_tc<256, kActNone, true>(probs, n_probs, dev_status, stream);
+  if (bn == 192) return pair ? run_tc_pair<192, kActNone, true>(probs, n_probs, dev_status, stream)
+                             : run_tc<192, kActNone, true>(probs, n_probs, dev_status, stream);
+  return pair ? run_tc_pair<128, kActNone, true>(probs, n_probs, dev_status, stream)
+              : run_tc<128, kActNone, true>(probs, n_probs, dev_status, stream);
 }
 
 }  // namespace moe

@@ -3,6 +3,7 @@
 // moe_status, and never synchronises the host.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -51,6 +52,8 @@ struct DispatchArgs {
   const int32_t *sel;
   int32_t *offsets, *perm, *row_of, *tok_ptr, *tok_assign;
   int32_t *dev_status;
+  int32_t *zero_words;  // optional: words the dispatch clears for a later kernel
+  int n_zero_words;
 };
 size_t dispatch_workspace_bytes(int64_t n_assign, int n_heavy);
 int launch_dispatch(const DispatchArgs &a, void *ws, cudaStream_t stream);
@@ -83,9 +86,26 @@ int launch_grouped_gemm_bf16(const GemmProblem *probs, int n_probs, int act,
                              bool out_f32, int32_t *dev_status,
                              cudaStream_t stream);
 
+// 2-D bf16 TMA descriptor [rows, cols] (cols contiguous), box {64, box_rows},
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_tma_2d_bf16(CUtensorMap *map, const void *ptr, int64_t rows, int64_t cols, int box_rows);
+
+// stream_sm100.cu: weight-streaming expert MLP for blocks of at most 128
+// tokens (each expert's weights read from HBM once per layer).
+bool stream_mlp_supported(int T);
+size_t stream_mlp_workspace_bytes(int n_groups);
+// `done` holds n_groups zeroed counters when counters_zeroed, else the
+// launcher clears them first.
+int launch_stream_mlp(const GemmProblem &up, int act, const GemmProblem &down,
+                      int max_tokens, int32_t *done, bool counters_zeroed,
+                      int32_t *dev_status, cudaStream_t stream);
+
 // mlp_f32.cu: the same grouped GEMM in fp32 on CUDA cores (fp32 layers).
 int launch_grouped_gemm_f32(const GemmProblem &p, int act,
                             cudaStream_t stream);
+
+// activation.cu: the experts' elementwise activation on its own.
+int launch_activation(const float *x, float *y, int64_t n, int act, cudaStream_t stream);
 
 // combine.cu
 struct CombineArgs {

@@ -82,7 +82,7 @@ int n_const_of(const moe_config &c) {
 // Workspace layout shared by the entry points.
 struct Layout {
   size_t logits, probs, sel, w, votes, core, offsets, perm, row_of, tok_ptr, tok_assign, dpart,
-      x_perm, H, H_sh, Y, Y_sh, x_dev, res_dev, zp_dev, y_dev, total;
+      x_perm, H, H_sh, Y, Y_sh, done, x_dev, res_dev, zp_dev, y_dev, total;
 };
 
 Layout layout_of(const moe_config &c) {
@@ -110,6 +110,7 @@ Layout layout_of(const moe_config &c) {
   L.H_sh = take((size_t)c.T * hs * eb);
   L.Y = take((size_t)na * c.d * 4);
   L.Y_sh = take(hs ? (size_t)c.T * c.d * 4 : 0);
+  L.done = take(stream_mlp_workspace_bytes(c.n_heavy + 1));  // routed groups, then the shared one
   L.x_dev = take((size_t)c.T * c.d * eb);
   L.res_dev = take((size_t)c.T * c.d * eb);
   L.zp_dev = take((size_t)c.T * c.E * 4);
@@ -132,7 +133,8 @@ int check_ws(const moe_config &c, void *ws, size_t ws_bytes) {
 int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offsets,
                     const void *W1, const void *W2, const void *x, const void *Ws1,
                     const void *Ws2, float *y_perm, float *y_shared, int32_t *dev_status,
-                    void *ws, const Layout &L, cudaStream_t stream) {
+                    void *ws, const Layout &L, cudaStream_t stream,
+                    bool counters_zeroed = false) {
   const int64_t na = n_assign_of(c);
   const int64_t hs = (int64_t)c.n_shared * c.h_shared;
   void *H = at<void>(ws, L.H);
@@ -153,6 +155,17 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
   const bool shared = hs > 0 && c.T > 0;
 
   int st = MOE_OK;
+  if (c.dtype == MOE_BF16 && stream_mlp_supported(c.T)) {
+    // Small blocks (every expert serves <= T <= 128 tokens): stream each
+    // used expert's weights once through the tensor cores.
+    int32_t *done = at<int32_t>(ws, L.done);
+    if (routed)
+      st = launch_stream_mlp(g1r, act1, g2r, c.T, done, counters_zeroed, dev_status, stream);
+    if (st == MOE_OK && shared)
+      st = launch_stream_mlp(g1s, kActGelu, g2s, c.T, done + c.n_heavy, counters_zeroed,
+                             dev_status, stream);
+    return st;
+  }
   if (c.dtype == MOE_BF16) {
     // GEMM1 (+activation): routed and shared in one tile stream when they share the activation.
     if (routed && shared && act1 == kActGelu) {
@@ -195,6 +208,7 @@ DispatchArgs dispatch_args(const moe_config &c, const int32_t *sel, int32_t *off
   a.n_assign = n_assign_of(c);
   a.sel = sel; a.offsets = offsets; a.perm = perm; a.row_of = row_of;
   a.tok_ptr = tok_ptr; a.tok_assign = tok_assign; a.dev_status = dev_status;
+  a.zero_words = nullptr; a.n_zero_words = 0;
   return a;
 }
 
@@ -243,13 +257,19 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
   if (st != MOE_OK) return st;
 
   DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
+  const bool streaming = c.dtype == MOE_BF16 && stream_mlp_supported(c.T);
+  if (streaming) {  // the dispatch clears the weight-streaming kernel's counters
+    da.zero_words = at<int32_t>(ws, L.done);
+    da.n_zero_words = c.n_heavy + 1;
+  }
   st = launch_dispatch(da, at<void>(ws, L.dpart), stream);
   if (st != MOE_OK) return st;
   if (c.n_heavy > 0) {
     st = launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, na, c.d, elem_bytes(c.dtype), stream);
     if (st != MOE_OK) return st;
   }
-  st = run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, Y, Y_sh, dev_status, ws, L, stream);
+  st = run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, Y, Y_sh, dev_status, ws, L, stream,
+                       streaming);
   if (st != MOE_OK) return st;
   CombineArgs ca = combine_args(c, Y, Y_sh, sel, w, row_of, tok_ptr, tok_assign, x, const_vecs,
                                 residual, y, dev_status);
@@ -429,6 +449,12 @@ int moe_combine(const moe_config *cfg, const float *y_perm, const float *y_share
   CombineArgs ca = combine_args(c, y_perm, c.n_shared > 0 ? y_shared : nullptr, sel, w, row_of,
                                 tok_ptr, tok_assign, x, const_vecs, residual, y, dev_status);
   return launch_combine(ca, kind_table(c), stream);
+}
+
+int moe_activation(const float *x, float *y, int64_t n, int act, moe_stream_t stream) {
+  if (n < 0 || (act != MOE_GELU_ERF && act != MOE_SWIGLU)) return MOE_ERR_INVALID_ARG;
+  if (n > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
+  return launch_activation(x, y, n, act, stream);
 }
 
 int moe_forward(const moe_config *cfg, const void *x, const void *residual, const float *z_prev,

@@ -31,6 +31,7 @@ constexpr int kBK = 64;        // model-width slice per pipeline stage
 constexpr int kLDS = kBK + 8;  // padded smem row (bf16): conflict-free ldmatrix
 constexpr int kStages = 3;
 constexpr int kThreads = 128;
+constexpr int kRowwiseMaxTokens = 512;  // bf16 layers this small use one CTA per token
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
   uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -264,6 +265,78 @@ router_f32_kernel(const float *__restrict__ x, const float *__restrict__ Wr,
   }
 }
 
+// Small blocks: one CTA per token, 8 warps sharing the E dot products of
+// length d (16-byte loads of the x row and of W_r rows), then warp 0
+// finishes softmax and top-k. Latency-bound; used when T is small enough
+// that a 64-token MMA tile would leave most of the GPU idle.
+constexpr int kRowThreads = 256;
+template <int VPL>
+__global__ void __launch_bounds__(kRowThreads)
+router_rowwise_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Wr,
+                           const float *__restrict__ bias, const float *__restrict__ zprev,
+                           float zscale, int T, int d, int E, float *__restrict__ logits,
+                           float *__restrict__ probs, int k, int renorm,
+                           int32_t *__restrict__ idx, float *__restrict__ w) {
+  __shared__ float zs[32 * VPL];
+  const int s = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kRowThreads / 32;
+  constexpr int kEB = 8;  // experts per register block: their loads are issued together
+  const __nv_bfloat16 *xr = x + (size_t)s * d;
+  for (int e0 = warp * kEB; e0 < E; e0 += kWarps * kEB) {
+    float p[kEB];
+#pragma unroll
+    for (int j = 0; j < kEB; ++j) p[j] = 0.f;
+    const __nv_bfloat16 *w0 = Wr + (size_t)e0 * d;
+#pragma unroll 2
+    for (int c = lane * 8; c < d; c += 256) {
+      uint4 xa = *reinterpret_cast<const uint4 *>(xr + c);
+      uint4 wb[kEB];
+#pragma unroll
+      for (int j = 0; j < kEB; ++j)
+        wb[j] = (e0 + j < E) ? *reinterpret_cast<const uint4 *>(w0 + (size_t)j * d + c)
+                             : make_uint4(0, 0, 0, 0);
+      const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&xa);
+#pragma unroll
+      for (int j = 0; j < kEB; ++j) {
+        const __nv_bfloat162 *wh = reinterpret_cast<const __nv_bfloat162 *>(&wb[j]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 a = __bfloat1622float2(xh[i]), b = __bfloat1622float2(wh[i]);
+          p[j] = fmaf(a.x, b.x, p[j]);
+          p[j] = fmaf(a.y, b.y, p[j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kEB; ++j) {
+      const float t = warp_sum(p[j]);
+      if (lane == 0 && e0 + j < E) zs[e0 + j] = t;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  float z[VPL], A[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int e = lane + 32 * v;
+    float zz = -INFINITY;
+    if (e < E) {
+      zz = zs[e];
+      if (bias) zz += bias[e];
+      if (zprev) zz += zscale * zprev[(size_t)s * E + e];
+      logits[(size_t)s * E + e] = zz;
+    }
+    z[v] = zz;
+  }
+  row_softmax<VPL>(z, E, A);
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int e = lane + 32 * v;
+    if (e < E) probs[(size_t)s * E + e] = A[v];
+  }
+  if (k > 0) row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(kThreads)
 select_topk_kernel(const float *__restrict__ logits, const float *__restrict__ probs, int T,
@@ -313,6 +386,15 @@ int launch_router(const void *x, const void *W_r, const float *bias, const float
                   float *probs, int k, int renorm, int32_t *idx, float *w,
                   cudaStream_t stream) {
   if (T == 0) return MOE_OK;
+  if (dtype == MOE_BF16 && T <= kRowwiseMaxTokens) {
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+    const __nv_bfloat16 *wb = static_cast<const __nv_bfloat16 *>(W_r);
+    const int vpl = (E + 31) / 32;
+    if (vpl == 1) router_rowwise_bf16_kernel<1><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
+    else if (vpl == 2) router_rowwise_bf16_kernel<2><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
+    else router_rowwise_bf16_kernel<4><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
+    return last_launch_status();
+  }
   if (dtype == MOE_BF16) {
     const int nt = (E + 7) / 8;
     if (nt <= 1) return run_router_bf16<1>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, stream);

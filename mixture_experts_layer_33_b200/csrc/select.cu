@@ -123,15 +123,16 @@ expert_choice_kernel(const float *__restrict__ probs, int E, int S, int C,
   (void)lane;
 }
 
-constexpr int kDesThreads = 256;
-constexpr int kDesVpl = MOE_MAX_EXPERTS / 32;  // experts per lane (M <= 256)
+constexpr int kDesThreads = 1024;  // one warp per token of a 32-token block
 
 // q(p) = round-half-even(p * 2^40): exact in double, then rounded once.
 __device__ __forceinline__ long long vote_quantum(float p) {
   return __double2ll_rn((double)p * 1099511627776.0);
 }
 
-// One CTA for the whole block of N tokens.
+// One CTA for the whole block of N tokens; each lane holds kDesVpl of a
+// token's M <= 32*kDesVpl probabilities.
+template <int kDesVpl>
 __global__ void __launch_bounds__(kDesThreads)
 des_vote_kernel(const float *__restrict__ P, int N, int M, int K, int Mc,
                 int64_t *__restrict__ votes, int32_t *__restrict__ core,
@@ -241,7 +242,10 @@ int launch_expert_choice(const float *probs, int T, int E, int S, int C, int32_t
 
 int launch_des_vote(const float *probs, int N, int M, int K, int M_core, int64_t *votes,
                     int32_t *core, int32_t *idx, float *w, cudaStream_t stream) {
-  des_vote_kernel<<<1, kDesThreads, 0, stream>>>(probs, N, M, K, M_core, votes, core, idx, w);
+  if (M <= 32) des_vote_kernel<1><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, M_core, votes, core, idx, w);
+  else if (M <= 64) des_vote_kernel<2><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, M_core, votes, core, idx, w);
+  else if (M <= 128) des_vote_kernel<4><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, M_core, votes, core, idx, w);
+  else des_vote_kernel<8><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, M_core, votes, core, idx, w);
   return last_launch_status();
 }
 

@@ -30,7 +30,7 @@ ENTRY_POINTS = (
     "moe_workspace_size", "moe_router", "moe_select_topk",
     "moe_select_expert_choice", "moe_core_set_vote", "moe_dispatch",
     "moe_grouped_mlp", "moe_combine", "moe_forward", "moe_forward_host",
-    "moe_dispatch_noalloc",
+    "moe_dispatch_noalloc", "moe_activation",
 )
 NOALLOC_SCRATCH_BYTES = 256 * 1024  # MOE_NOALLOC_SCRATCH_BYTES
 
@@ -66,6 +66,7 @@ _SIGS = {
     "moe_core_set_vote": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_dispatch": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_dispatch_noalloc": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_activation": (_i32, [_vp, _vp, ctypes.c_int64, _i32, _vp]),
     "moe_grouped_mlp": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                _vp]),
     "moe_combine": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -228,6 +229,12 @@ def dispatch_noalloc(c: MoeConfig, sel, x, x_perm, offsets, perm, row_of, tok_pt
             f"(ceil(n_assign/1024) * n_heavy * 4 bytes) exceeds the {NOALLOC_SCRATCH_BYTES}-byte "
             "library-owned array; use dispatch() with a workspace")
     _check(code, "moe_dispatch_noalloc")
+
+
+def activation(x, y, act=GELU_ERF, stream=None):
+    """y = GELU(x) (act=GELU_ERF) or SiLU(x) (act=SWIGLU), fp32 device tensors."""
+    _check(LIB.moe_activation(_dev_ptr(x), _dev_ptr(y), x.numel(), int(act), _stream(stream)),
+           "moe_activation")
 
 
 def grouped_mlp(c: MoeConfig, x_perm, offsets, W1, W2, x, Ws1, Ws2, y_perm, y_shared,

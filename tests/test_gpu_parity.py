@@ -27,6 +27,12 @@ SMALL = [
     ("mmoe", dict(T=600, d=256, h=512, h_shared=256)),
     ("mmoe_skewed", dict(T=600, d=256, h=512, h_shared=256)),
 ]
+# Groups averaging >= 256 rows: the grouped GEMM runs on two-SM (M=256) tiles.
+PAIR = [
+    ("ditmoe_xl", dict(T=2048, d=256, h=512, h_shared=256)),
+    ("ecdit", dict(T=32 * 128, group_size=128, d=256, E=8, h=512, capacity=32)),
+    ("des_vote", dict(T=1024, d=256, E=16, k=4, h=256, M_core=8)),
+]
 FULL = ["tiny_fp32", "ditmoe_xl", "ecdit", "des_vote", "mmoe", "mmoe_skewed"]
 
 
@@ -58,6 +64,19 @@ def _check_selection(cfg, out):
 
 @pytest.mark.parametrize("name,over", SMALL, ids=[s[0] for s in SMALL])
 def test_layer_small_full_oracle(name, over):
+    cfg = gen.workload(name, **over)
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    assert out["status"] == 0
+    hin = H.host(inp)
+    _check_router(cfg, hin, out)
+    sel = _check_selection(cfg, out)
+    y_ref = H.oracle_layer(cfg, hin, sel)
+    assert H.normwise(out["y"], y_ref) <= H.Y_TOL[cfg["dtype"]]
+
+
+@pytest.mark.parametrize("name,over", PAIR, ids=[p[0] for p in PAIR])
+def test_layer_two_sm_tiles_full_oracle(name, over):
     cfg = gen.workload(name, **over)
     inp = gen.make_inputs(cfg, "cuda")
     out = H.run_layer(cfg, inp)
