@@ -8,7 +8,8 @@ dispatch -> grouped expert MLP -> combine) over one batch of synthetic input
 through moe_forward, replayed as a CUDA graph; a second timed loop issues
 the same layer as the staged C-ABI calls with a CUDA event between stages
 for the per-stage split and the grouped MLP's own duration. L2 is flushed
-(a 256 MiB write) before every timed step, outside the events. ``value`` is
+before every timed step, outside the events: a 256 MiB write, then a
+256 MiB read so no dirty flush data is left to write back. ``value`` is
 tokens/s over the K timed steps (inputs resident in HBM); ``e2e`` repeats
 the measurement through moe_forward_host with the activations in pinned
 host memory and the copies inside the timed region. Multi-GPU runs are
@@ -33,6 +34,22 @@ DEFAULT_WORKLOAD = "ditmoe_xl"
 METRIC = "MoE-layer tokens/s and TFLOP/s (or HBM GB/s) vs B200 roofline, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Leaves L2 cold and clean between timed steps: writes a 256 MiB buffer
+    (evicting everything) and then reads another (so the lines left behind
+    are clean and the timed step pays no write-back of the flush's own data).
+    Runs outside the timed events."""
+
+    def __init__(self, device):
+        import torch
+        self.a = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        self.b = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def __call__(self, step=0):
+        self.a.fill_(step & 255)
+        self.sink = self.b.sum()
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the grouped-MLP
 # launches of one layer pass, from one ncu capture (profiles/), valid only while
@@ -225,8 +242,8 @@ class StagedLayer:
         self.tok_ptr = torch.empty(T + 1, dtype=torch.int32, **f) if ec else None
         self.tok_assign = torch.empty(na, dtype=torch.int32, **f) if ec else None
         self.x_perm = torch.empty(na, d, dtype=inp["x"].dtype, **f)
-        self.y_perm = torch.empty(na, d, dtype=torch.float32, **f)
-        self.y_sh = torch.empty(T, d, dtype=torch.float32, **f) if cfg["n_shared"] else None
+        self.y_perm = torch.empty(na, d, dtype=inp["x"].dtype, **f)
+        self.y_sh = torch.empty(T, d, dtype=inp["x"].dtype, **f) if cfg["n_shared"] else None
         self.y = torch.empty_like(inp["x"])
         self.ws = m.alloc_workspace(self.c, device)
         self.status = torch.zeros(1, dtype=torch.int32, **f)
@@ -307,11 +324,11 @@ def gpu_bench(args):
     cfg = gen.workload(args.workload)
     inp = gen.make_inputs(cfg, dev)
     layer = StagedLayer(m, cfg, inp, dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
-        flush.fill_(1)
+        flush(1)
         layer.run()
     torch.cuda.synchronize()
     if int(layer.status.item()) != 0:
@@ -334,7 +351,7 @@ def gpu_bench(args):
             with torch.cuda.graph(graph):
                 layer.run_forward()
             for _ in range(3):
-                flush.fill_(1)
+                flush(1)
                 graph.replay()
             torch.cuda.synchronize()
         except Exception as exc:  # noqa: BLE001
@@ -350,7 +367,7 @@ def gpu_bench(args):
         dist.barrier()
     torch.cuda.synchronize()
     for s in range(args.steps):
-        flush.fill_(s & 255)
+        flush(s)
         ev[s][0].record()
         if graph is not None:
             graph.replay()
@@ -371,7 +388,7 @@ def gpu_bench(args):
     sev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     torch.cuda.synchronize()
     for s in range(args.steps):
-        flush.fill_(s & 255)
+        flush(s)
         layer.run(sev[s])
     torch.cuda.synchronize()
     stage_ms = {n: 0.0 for n in layer.stages}
@@ -395,7 +412,7 @@ def gpu_bench(args):
     torch.cuda.synchronize()
     e2e_ms = 0.0
     for s in range(args.steps):
-        flush.fill_(s & 255)
+        flush(s)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         e2e_step()
@@ -432,7 +449,7 @@ def gpu_bench(args):
         "dtype": cfg["dtype"], "data": "synthetic (seeded Gaussian inputs, random-init weights)",
         "config": {"workload": describe(cfg), "global_batch_tokens": cfg["T"] * world,
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "l2": "flushed by a 256 MiB write before every timed step"},
+                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so L2 is left clean)"},
         "layer_tflops": round(flops / (ms_per_step / 1e3) / 1e12, 1),
         "layer_weight_gbs": round(weight_bytes_used(cfg, used) / (ms_per_step / 1e3) / 1e9, 1),
         "cuda_graph": graph is not None,

@@ -258,14 +258,15 @@ MOE_API int moe_dispatch_noalloc(const moe_config *cfg, const int32_t *sel,
  *   W2      [n_heavy, d, h]
  *   x       [T, d], Ws1 [n_shared*h_shared, d], Ws2 [d, n_shared*h_shared]
  *           (all three nullable when n_shared == 0)
- *   y_perm  [n_assign, d] fp32 out: W2_e . act(W1_e . x_perm[r]) per row r
- *   y_shared [T, d] fp32 out (nullable when n_shared == 0)
- * Hidden activations are kept in `dtype` in the workspace.
+ *   y_perm  [n_assign, d] out (dtype): W2_e . act(W1_e . x_perm[r]) per row r
+ *   y_shared [T, d] out (dtype; nullable when n_shared == 0)
+ * Accumulation is fp32 in tensor memory; hidden activations and outputs are
+ * rounded to `dtype` (bf16 layers: bf16).
  */
 MOE_API int moe_grouped_mlp(const moe_config *cfg, const void *x_perm,
                     const int32_t *offsets, const void *W1, const void *W2,
                     const void *x, const void *Ws1, const void *Ws2,
-                    float *y_perm, float *y_shared, int32_t *dev_status,
+                    void *y_perm, void *y_shared, int32_t *dev_status,
                     void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
@@ -275,14 +276,16 @@ MOE_API int moe_grouped_mlp(const moe_config *cfg, const void *x_perm,
  *   y_s = r_s + y_shared[s] + sum over s's assignments a (in slot order) of
  *         w[a] * { y_perm[row_of[a]] (heavy), x_s (identity), 0 (zero),
  *                  const_vecs[c] (c-th constant expert) }
- * summed in fp32 and rounded once to dtype.
+ * summed in fp32 and rounded once to dtype. y_perm, y_shared are in dtype.
+ * `residual` may be the same buffer as `y` (the sum is formed element by
+ * element before y is written).
  *   sel, w       the selection (as in moe_dispatch) and its [n_assign] weights
  *   row_of       from moe_dispatch;  tok_ptr/tok_assign: expert choice only
  *   x            [T, d] (identity experts); const_vecs [n_const, d], nullable
  *   residual     [T, d] nullable (r = 0);  y [T, d] out (dtype)
  */
-MOE_API int moe_combine(const moe_config *cfg, const float *y_perm,
-                const float *y_shared, const int32_t *sel, const float *w,
+MOE_API int moe_combine(const moe_config *cfg, const void *y_perm,
+                const void *y_shared, const int32_t *sel, const float *w,
                 const int32_t *row_of, const int32_t *tok_ptr,
                 const int32_t *tok_assign, const void *x,
                 const void *const_vecs, const void *residual, void *y,

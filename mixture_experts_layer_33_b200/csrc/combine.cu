@@ -11,8 +11,10 @@
 //
 // One warp per (token, 256-feature chunk); each lane owns 8 consecutive
 // features and reads them with 16-byte loads; a token's slot metadata is
-// loaded once, one slot per lane, and broadcast by shuffles. The sum runs in fp32 in slot order (no
-// atomics, so the output is bitwise deterministic) and is rounded once.
+// loaded once, one slot per lane, and broadcast by shuffles. Expert outputs
+// arrive in the layer dtype; the sum runs in fp32 in slot order (no atomics,
+// so the output is bitwise deterministic) and is rounded once. `residual`
+// may alias `y` (the forward pass writes x + shared(x) into y first).
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,10 +26,11 @@ constexpr int kThreads = 256;
 template <typename T>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTable kinds) {
   const T *__restrict__ x = static_cast<const T *>(a.x);
-  const T *__restrict__ res = static_cast<const T *>(a.residual);
+  const T *res = static_cast<const T *>(a.residual);  // may alias y
   const T *__restrict__ cv = static_cast<const T *>(a.const_vecs);
-  const float *__restrict__ yp = a.y_perm;
-  T *__restrict__ y = static_cast<T *>(a.y);
+  const T *__restrict__ yp = static_cast<const T *>(a.y_perm);
+  const T *__restrict__ ysh = static_cast<const T *>(a.y_shared);
+  T *y = static_cast<T *>(a.y);
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * kThreads + threadIdx.x) >> 5;
   const int nw = (gridDim.x * kThreads) >> 5;
@@ -46,9 +49,9 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     if (live && res) load8(res + (size_t)s * a.d + c0, acc);
-    if (live && a.y_shared) {
+    if (live && ysh) {
       float t[8];
-      load8(a.y_shared + (size_t)s * a.d + c0, t);
+      load8(ysh + (size_t)s * a.d + c0, t);
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += t[i];
     }

@@ -151,6 +151,13 @@ __device__ __forceinline__ float gelu_erf(float v) {
 // SiLU(u) = u / (1 + exp(-u)), with the accurate expf (a few ulps at any u).
 __device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.0f + expf(-v)); }
 
+// DES-Vote fixed point: q(p) = round-half-even(p * 2^40) as int64. The
+// product is exact in double and rounded once, so integer sums of votes
+// are exact and independent of the order they are added in.
+__device__ __forceinline__ long long vote_quantum(float p) {
+  return __double2ll_rn((double)p * 1099511627776.0);
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -51,6 +51,8 @@ struct ProbDev {
   void *out;
   int64_t ld_out;
   int vec32;  // rows of `out` start on 32-byte boundaries: 256-bit stores
+  const __nv_bfloat16 *residual;  // optional, added before rounding (bf16 outputs)
+  int64_t ld_res;
 };
 struct ParamsDev {
   int n_probs;
@@ -109,11 +111,28 @@ __device__ __forceinline__ void store_row32(const ProbDev &pr, int row, int col,
     }
   } else {
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(pr.out) + (int64_t)row * pr.ld_out + col;
+    float r[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = 0.f;
+    if (pr.residual) {
+      const __nv_bfloat16 *rp = pr.residual + (int64_t)row * pr.ld_res + col;
+      if (col + 32 <= pr.N) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          float t[8];
+          load8(rp + i, t);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) r[i + j] = t[j];
+        }
+      } else {
+        for (int i = 0; i < 32 && col + i < pr.N; ++i) r[i] = __bfloat162float(rp[i]);
+      }
+    }
     if (col + 32 <= pr.N) {
       uint32_t w[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j] + r[2 * j], v[2 * j + 1] + r[2 * j + 1]);
         w[j] = *reinterpret_cast<uint32_t *>(&h2);
       }
       if (pr.vec32) {
@@ -125,7 +144,7 @@ __device__ __forceinline__ void store_row32(const ProbDev &pr, int row, int col,
           *reinterpret_cast<uint4 *>(o + 8 * i) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
       }
     } else {
-      for (int i = 0; i < 32 && col + i < pr.N; ++i) o[i] = __float2bfloat16_rn(v[i]);
+      for (int i = 0; i < 32 && col + i < pr.N; ++i) o[i] = __float2bfloat16_rn(v[i] + r[i]);
     }
   }
 }
@@ -631,6 +650,8 @@ int run_tc(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t 
     pd.pr[i].out = q.out;
     pd.pr[i].ld_out = q.ld_out;
     pd.pr[i].vec32 = vec32_ok(q, OUT_F32 ? 4 : 2);
+    pd.pr[i].residual = static_cast<const __nv_bfloat16 *>(q.residual);
+    pd.pr[i].ld_res = q.ld_res;
     max_tiles += max_m_tiles(q, BM) * ((q.N + BNO - 1) / BNO);
   }
   if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; }
@@ -672,6 +693,8 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
     pd.pr[i].out = q.out;
     pd.pr[i].ld_out = q.ld_out;
     pd.pr[i].vec32 = vec32_ok(q, OUT_F32 ? 4 : 2);
+    pd.pr[i].residual = static_cast<const __nv_bfloat16 *>(q.residual);
+    pd.pr[i].ld_res = q.ld_res;
     max_tiles += max_m_tiles(q, 2 * BM) * ((q.N + BNO - 1) / BNO);
   }
   if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; }
@@ -737,32 +760,28 @@ static bool use_pair(const GemmProblem *probs, int n_probs, int bn) {
 int launch_grouped_gemm_bf16(const GemmProblem *probs, int n_probs, int act, bool out_f32,
                              int32_t *dev_status, cudaStream_t stream) {
   if (n_probs < 1 || n_probs > 2) return MOE_ERR_INVALID_ARG;
+  if (out_f32) return MOE_ERR_UNSUPPORTED;  // bf16 layers keep every GEMM output in bf16
   const int bn = pick_bn(probs, n_probs, act);
   const bool pair = use_pair(probs, n_probs, bn);
-  if (!out_f32) {
-    if (act == kActGelu) {
-      if (bn == 256) return pair ? run_tc_pair<256, kActGelu, false>(probs, n_probs, dev_status, stream)
-                                 : run_tc<256, kActGelu, false>(probs, n_probs, dev_status, stream);
-      if (bn == 192) return pair ? run_tc_pair<192, kActGelu, false>(probs, n_probs, dev_status, stream)
-                                 : run_tc<192, kActGelu, false>(probs, n_probs, dev_status, stream);
-      return pair ? run_tc_pair<128, kActGelu, false>(probs, n_probs, dev_status, stream)
-                  : run_tc<128, kActGelu, false>(probs, n_probs, dev_status, stream);
-    }
-    if (act == kActSwiglu) {
-      if (bn == 256) return pair ? run_tc_pair<256, kActSwiglu, false>(probs, n_probs, dev_status, stream)
-                                 : run_tc<256, kActSwiglu, false>(probs, n_probs, dev_status, stream);
-      return pair ? run_tc_pair<128, kActSwiglu, false>(probs, n_probs, dev_status, stream)
-                  : run_tc<128, kActSwiglu, false>(probs, n_probs, dev_status, stream);
-    }
-    return MOE_ERR_UNSUPPORTED;
+#define MOE_RUN(BN_, ACT_) \
+  return pair ? run_tc_pair<BN_, ACT_, false>(probs, n_probs, dev_status, stream) \
+              : run_tc<BN_, ACT_, false>(probs, n_probs, dev_status, stream)
+  if (act == kActGelu) {
+    if (bn == 256) MOE_RUN(256, kActGelu);
+    if (bn == 192) MOE_RUN(192, kActGelu);
+    MOE_RUN(128, kActGelu);
   }
-  if (act != kActNone) return MOE_ERR_UNSUPPORTED;
-  if (bn == 256) return pair ? run_tc_pair<256, kActNone, true>(probs, n_probs, dev_status, stream)
-                             : run_tc<256, kActNone, true>(probs, n_probs, dev_status, stream);
-  if (bn == 192) return pair ? run_tc_pair<192, kActNone, true>(probs, n_probs, dev_status, stream)
-                             : run_tc<192, kActNone, true>(probs, n_probs, dev_status, stream);
-  return pair ? run_tc_pair<128, kActNone, true>(probs, n_probs, dev_status, stream)
-              : run_tc<128, kActNone, true>(probs, n_probs, dev_status, stream);
+  if (act == kActSwiglu) {
+    if (bn == 256) MOE_RUN(256, kActSwiglu);
+    MOE_RUN(128, kActSwiglu);
+  }
+  if (act == kActNone) {
+    if (bn == 256) MOE_RUN(256, kActNone);
+    if (bn == 192) MOE_RUN(192, kActNone);
+    MOE_RUN(128, kActNone);
+  }
+#undef MOE_RUN
+  return MOE_ERR_UNSUPPORTED;
 }
 
 }  // namespace moe

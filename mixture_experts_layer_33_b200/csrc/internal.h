@@ -27,10 +27,22 @@ inline int last_launch_status() {
 int num_sms();
 
 // router.cu: z = x W_r^T + bias + scale * z_prev; A = softmax(z); optional top-k.
+// With `votes` (zeroed int64 [E]) the router also adds each token's DES
+// top-k_vote votes into it (small bf16 blocks only: router_can_vote).
 int launch_router(const void *x, const void *W_r, const float *bias,
                   const float *z_prev, float z_prev_scale, int T, int d, int E,
                   int dtype, float *logits, float *probs, int k, int renorm,
-                  int32_t *idx, float *w, cudaStream_t stream);
+                  int32_t *idx, float *w, cudaStream_t stream,
+                  int64_t *votes = nullptr, int k_vote = 0);
+bool router_can_vote(int T, int dtype);
+// Small bf16 blocks in the fused forward: the model width is split over
+// n_part CTAs per 32-token tile (partial logits in `part`, [n_part][T][E]
+// fp32), then one warp per token finishes (and optionally votes).
+int router_split_parts(int T, int d, int dtype);  // 0: not used for this size
+int launch_router_split(const void *x, const void *W_r, const float *bias, const float *z_prev,
+                        float z_prev_scale, int T, int d, int E, float *part, int n_part,
+                        float *logits, float *probs, int k, int renorm, int32_t *idx, float *w,
+                        int64_t *votes, int k_vote, cudaStream_t stream);
 int launch_select_topk(const float *logits, const float *probs, int T, int E,
                        int k, int renorm, int32_t *idx, float *w,
                        cudaStream_t stream);
@@ -38,6 +50,10 @@ int launch_select_topk(const float *logits, const float *probs, int T, int E,
 // select.cu: expert-choice radix select and the DES-Vote core set.
 int launch_expert_choice(const float *probs, int T, int E, int S, int C,
                          int32_t *tok, float *w, cudaStream_t stream);
+// Election recomputed per token-CTA from summed votes, then re-routing.
+int launch_des_reroute(const float *probs, const int64_t *votes, int N, int M, int K,
+                       int M_core, int32_t *core, int32_t *idx, float *w,
+                       cudaStream_t stream);
 int launch_des_vote(const float *probs, int N, int M, int K, int M_core,
                     int64_t *votes, int32_t *core, int32_t *idx, float *w,
                     cudaStream_t stream);
@@ -76,6 +92,8 @@ struct GemmProblem {
   int N, K;
   void *out;            // [rows, ld_out] (bf16 or fp32)
   int64_t ld_out;
+  const void *residual; // optional [rows, ld_res] bf16 added before the output is rounded
+  int64_t ld_res;
 };
 
 // Upper bound of the m-tiles of height bm over all groups of a problem.
@@ -110,7 +128,7 @@ int launch_activation(const float *x, float *y, int64_t n, int act, cudaStream_t
 // combine.cu
 struct CombineArgs {
   int routing, T, d, E, k, S, C, dtype;
-  const float *y_perm, *y_shared;
+  const void *y_perm, *y_shared;  // expert outputs, in the layer dtype
   const int32_t *sel;
   const float *w;
   const int32_t *row_of, *tok_ptr, *tok_assign;

@@ -82,7 +82,7 @@ int n_const_of(const moe_config &c) {
 // Workspace layout shared by the entry points.
 struct Layout {
   size_t logits, probs, sel, w, votes, core, offsets, perm, row_of, tok_ptr, tok_assign, dpart,
-      x_perm, H, H_sh, Y, Y_sh, done, x_dev, res_dev, zp_dev, y_dev, total;
+      x_perm, H, H_sh, Y, Y_sh, done, rpart, x_dev, res_dev, zp_dev, y_dev, total;
 };
 
 Layout layout_of(const moe_config &c) {
@@ -108,9 +108,10 @@ Layout layout_of(const moe_config &c) {
   L.x_perm = take((size_t)na * c.d * eb);
   L.H = take((size_t)na * h1 * eb);
   L.H_sh = take((size_t)c.T * hs * eb);
-  L.Y = take((size_t)na * c.d * 4);
-  L.Y_sh = take(hs ? (size_t)c.T * c.d * 4 : 0);
+  L.Y = take((size_t)na * c.d * eb);
+  L.Y_sh = take(hs ? (size_t)c.T * c.d * eb : 0);
   L.done = take(stream_mlp_workspace_bytes(c.n_heavy + 1));  // routed groups, then the shared one
+  L.rpart = take((size_t)router_split_parts(c.T, c.d, c.dtype) * c.T * c.E * 4);
   L.x_dev = take((size_t)c.T * c.d * eb);
   L.res_dev = take((size_t)c.T * c.d * eb);
   L.zp_dev = take((size_t)c.T * c.E * 4);
@@ -132,9 +133,9 @@ int check_ws(const moe_config &c, void *ws, size_t ws_bytes) {
 
 int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offsets,
                     const void *W1, const void *W2, const void *x, const void *Ws1,
-                    const void *Ws2, float *y_perm, float *y_shared, int32_t *dev_status,
+                    const void *Ws2, void *y_perm, void *y_shared, int32_t *dev_status,
                     void *ws, const Layout &L, cudaStream_t stream,
-                    bool counters_zeroed = false) {
+                    bool counters_zeroed = false, const void *shared_residual = nullptr) {
   const int64_t na = n_assign_of(c);
   const int64_t hs = (int64_t)c.n_shared * c.h_shared;
   void *H = at<void>(ws, L.H);
@@ -151,6 +152,7 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
   g1s.N = (int)hs; g1s.b_rows_per_group = (int)hs; g1s.K = c.d; g1s.out = H_sh; g1s.ld_out = hs;
   g2s.A = H_sh; g2s.a_rows = c.T; g2s.B = Ws2; g2s.n_groups = 1; g2s.offsets = nullptr;
   g2s.N = c.d; g2s.b_rows_per_group = c.d; g2s.K = (int)hs; g2s.out = y_shared; g2s.ld_out = c.d;
+  g2s.residual = shared_residual; g2s.ld_res = c.d;
   const bool routed = c.n_heavy > 0 && na > 0;
   const bool shared = hs > 0 && c.T > 0;
 
@@ -179,11 +181,11 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
     // GEMM2: the longer-K shared problem first so the tile stream ends on short tiles.
     if (routed && shared) {
       GemmProblem p2[2] = {g2s, g2r};
-      st = launch_grouped_gemm_bf16(p2, 2, kActNone, true, dev_status, stream);
+      st = launch_grouped_gemm_bf16(p2, 2, kActNone, false, dev_status, stream);
     } else if (routed) {
-      st = launch_grouped_gemm_bf16(&g2r, 1, kActNone, true, dev_status, stream);
+      st = launch_grouped_gemm_bf16(&g2r, 1, kActNone, false, dev_status, stream);
     } else if (shared) {
-      st = launch_grouped_gemm_bf16(&g2s, 1, kActNone, true, dev_status, stream);
+      st = launch_grouped_gemm_bf16(&g2s, 1, kActNone, false, dev_status, stream);
     }
     return st;
   }
@@ -212,7 +214,7 @@ DispatchArgs dispatch_args(const moe_config &c, const int32_t *sel, int32_t *off
   return a;
 }
 
-CombineArgs combine_args(const moe_config &c, const float *y_perm, const float *y_shared,
+CombineArgs combine_args(const moe_config &c, const void *y_perm, const void *y_shared,
                          const int32_t *sel, const float *w, const int32_t *row_of,
                          const int32_t *tok_ptr, const int32_t *tok_assign, const void *x,
                          const void *const_vecs, const void *residual, void *y,
@@ -242,20 +244,35 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
   int32_t *tok_ptr = at<int32_t>(ws, L.tok_ptr), *tok_assign = at<int32_t>(ws, L.tok_assign);
   const int64_t na = n_assign_of(c);
   const int64_t hs = (int64_t)c.n_shared * c.h_shared;
-  float *Y = at<float>(ws, L.Y);
-  float *Y_sh = hs ? at<float>(ws, L.Y_sh) : nullptr;
+  void *Y = at<void>(ws, L.Y);
+  void *Y_sh = hs ? at<void>(ws, L.Y_sh) : nullptr;
   void *x_perm = at<void>(ws, L.x_perm);
 
-  int st = launch_router(x, W_r, bias, z_prev, c.gate_residual_scale, c.T, c.d, c.E, c.dtype,
-                         logits, probs, c.routing == MOE_TOKEN_TOPK ? c.k : 0, c.renorm, sel, w,
-                         stream);
-  if (st != MOE_OK) return st;
-  if (c.routing == MOE_EXPERT_CHOICE)
-    st = launch_expert_choice(probs, c.T, c.E, c.group_size, c.capacity, sel, w, stream);
-  else if (c.routing == MOE_DES_VOTE)
-    st = launch_des_vote(probs, c.T, c.E, c.k, c.M_core, votes, core, sel, w, stream);
-  if (st != MOE_OK) return st;
-
+  int st = MOE_OK;
+  const int n_part = router_split_parts(c.T, c.d, c.dtype);
+  if (n_part > 0 && c.routing != MOE_EXPERT_CHOICE) {
+    // Small bf16 block: router split over the model width, then a per-token
+    // finish that also selects (token choice) or sums the exact int64 DES
+    // votes; DES then elects the core set and re-routes per token.
+    const bool des = c.routing == MOE_DES_VOTE;
+    if (des) MOE_CUDA_TRY(cudaMemsetAsync(votes, 0, (size_t)c.E * sizeof(int64_t), stream));
+    st = launch_router_split(x, W_r, bias, z_prev, c.gate_residual_scale, c.T, c.d, c.E,
+                             at<float>(ws, L.rpart), n_part, logits, probs, des ? 0 : c.k,
+                             c.renorm, des ? nullptr : sel, des ? nullptr : w,
+                             des ? votes : nullptr, des ? c.k : 0, stream);
+    if (st == MOE_OK && des)
+      st = launch_des_reroute(probs, votes, c.T, c.E, c.k, c.M_core, core, sel, w, stream);
+    if (st != MOE_OK) return st;
+  } else {
+    st = launch_router(x, W_r, bias, z_prev, c.gate_residual_scale, c.T, c.d, c.E, c.dtype, logits,
+                       probs, c.routing == MOE_TOKEN_TOPK ? c.k : 0, c.renorm, sel, w, stream);
+    if (st != MOE_OK) return st;
+    if (c.routing == MOE_EXPERT_CHOICE)
+      st = launch_expert_choice(probs, c.T, c.E, c.group_size, c.capacity, sel, w, stream);
+    else if (c.routing == MOE_DES_VOTE)
+      st = launch_des_vote(probs, c.T, c.E, c.k, c.M_core, votes, core, sel, w, stream);
+    if (st != MOE_OK) return st;
+  }
   DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
   const bool streaming = c.dtype == MOE_BF16 && stream_mlp_supported(c.T);
   if (streaming) {  // the dispatch clears the weight-streaming kernel's counters
@@ -268,11 +285,16 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
     st = launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, na, c.d, elem_bytes(c.dtype), stream);
     if (st != MOE_OK) return st;
   }
-  st = run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, Y, Y_sh, dev_status, ws, L, stream,
-                       streaming);
+  // bf16 grouped-GEMM path with a shared expert: its down-projection epilogue
+  // writes y = residual + shared(x) straight into y, and the combine then adds
+  // the routed terms in place (no shared-output buffer round trip).
+  const bool shared_into_y = hs > 0 && c.dtype == MOE_BF16 && !streaming && c.T > 0;
+  st = run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, Y, shared_into_y ? y : Y_sh,
+                       dev_status, ws, L, stream, streaming, shared_into_y ? residual : nullptr);
   if (st != MOE_OK) return st;
-  CombineArgs ca = combine_args(c, Y, Y_sh, sel, w, row_of, tok_ptr, tok_assign, x, const_vecs,
-                                residual, y, dev_status);
+  CombineArgs ca = combine_args(c, Y, shared_into_y ? nullptr : Y_sh, sel, w, row_of, tok_ptr,
+                                tok_assign, x, const_vecs, shared_into_y ? y : residual, y,
+                                dev_status);
   return launch_combine(ca, kind_table(c), stream);
 }
 
@@ -414,7 +436,7 @@ int moe_dispatch_noalloc(const moe_config *cfg, const int32_t *sel, const void *
 
 int moe_grouped_mlp(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
                     const void *W1, const void *W2, const void *x, const void *Ws1,
-                    const void *Ws2, float *y_perm, float *y_shared, int32_t *dev_status,
+                    const void *Ws2, void *y_perm, void *y_shared, int32_t *dev_status,
                     void *ws, size_t ws_bytes, moe_stream_t stream) {
   int st = check_config(cfg);
   if (st != MOE_OK) return st;
@@ -430,7 +452,7 @@ int moe_grouped_mlp(const moe_config *cfg, const void *x_perm, const int32_t *of
                          ws, layout_of(c), stream);
 }
 
-int moe_combine(const moe_config *cfg, const float *y_perm, const float *y_shared,
+int moe_combine(const moe_config *cfg, const void *y_perm, const void *y_shared,
                 const int32_t *sel, const float *w, const int32_t *row_of,
                 const int32_t *tok_ptr, const int32_t *tok_assign, const void *x,
                 const void *const_vecs, const void *residual, void *y, int32_t *dev_status,

@@ -9,13 +9,16 @@
 // EC-DiT section 3 "Token-Choice routing": each token keeps its top-k
 // experts.
 //
-// bf16 path: a CTA owns 64 tokens; its 4 warps each run m16n8k16 bf16
-// tensor-core MMAs (fp32 accumulate) over cp.async-staged tiles of x and
-// W_r, so x is read from HBM exactly once. The N dimension of this GEMM is
-// E <= 128, far too narrow for a 128-wide tcgen05 tile; the kernel is bound
-// by reading x. The logits tile is then parked in shared memory and each
-// warp finishes its 16 tokens with warp-shuffle softmax and warp-shuffle
-// argmax rounds for the top-k (ties to the lower expert id).
+// bf16 path: a CTA owns 32 tokens; its 2 warps each run m16n8k16 bf16
+// tensor-core MMAs (fp32 accumulate) over a 6-deep cp.async ring of x and
+// W_r tiles, so x is read from HBM exactly once with many tiles in flight.
+// The N dimension of this GEMM is E <= 128, far too narrow for a 128-wide
+// tcgen05 tile; the kernel is bound by reading x. The logits tile is then
+// parked in shared memory; for E <= 32 each thread finishes one token's
+// softmax and top-k serially, for wider E each warp finishes its tokens
+// with warp-shuffle softmax and warp-shuffle argmax rounds (ties to the
+// lower expert id either way). Small blocks (T <= 512) use one CTA per
+// token instead, with 8 warps sharing the E dot products.
 // fp32 path: plain FMA dot products, one warp per token (fp32 layers are
 // small and must stay exact to fp32 rounding).
 #include <math.h>
@@ -32,6 +35,9 @@ constexpr int kLDS = kBK + 8;  // padded smem row (bf16): conflict-free ldmatrix
 constexpr int kStages = 3;
 constexpr int kThreads = 128;
 constexpr int kRowwiseMaxTokens = 512;  // bf16 layers this small use one CTA per token
+constexpr int kMmaBM = 32;               // tokens per CTA of the MMA router (2 warps x 16)
+constexpr int kMmaThreads = 64;
+constexpr int kMmaStages = 6;            // cp.async ring depth: many x tiles in flight per SM
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
   uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -115,8 +121,10 @@ __device__ __forceinline__ void row_topk(const float (&z)[VPL], const float (&A)
     for (int r = 0; r < k; ++r) w_row[r] = w_row[r] / wsum;
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kThreads)
+// PARTIAL: blockIdx.y selects a slice of the model width; the CTA writes
+// its partial logits to `logits` laid out [gridDim.y][T][E] and stops.
+template <int NT, bool PARTIAL = false>
+__global__ void __launch_bounds__(kMmaThreads)
 router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Wr,
                    const float *__restrict__ bias, const float *__restrict__ zprev, float zscale,
                    int T, int d, int E, float *__restrict__ logits, float *__restrict__ probs,
@@ -124,23 +132,26 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
   constexpr int EP = NT * 8;
   constexpr int VPL = (EP + 31) / 32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __nv_bfloat16 *sX = reinterpret_cast<__nv_bfloat16 *>(smem_raw);   // [stages][kBM][kLDS]
-  __nv_bfloat16 *sW = sX + kStages * kBM * kLDS;                      // [stages][EP][kLDS]
-  float *sZ = reinterpret_cast<float *>(sW + kStages * EP * kLDS);    // [kBM][EP + 1]
+  __nv_bfloat16 *sX = reinterpret_cast<__nv_bfloat16 *>(smem_raw);   // [stages][kMmaBM][kLDS]
+  __nv_bfloat16 *sW = sX + kMmaStages * kMmaBM * kLDS;                      // [stages][EP][kLDS]
+  float *sZ = reinterpret_cast<float *>(sW + kMmaStages * EP * kLDS);    // [kMmaBM][EP + 1]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * kBM;
-  const int nk = (d + kBK - 1) / kBK;
+  const int t0 = blockIdx.x * kMmaBM;
+  const int nk_all = (d + kBK - 1) / kBK;
+  const int kb_per = PARTIAL ? (nk_all + gridDim.y - 1) / gridDim.y : nk_all;
+  const int kb0 = PARTIAL ? blockIdx.y * kb_per : 0;
+  const int nk = PARTIAL ? max(0, min(nk_all, kb0 + kb_per) - kb0) : nk_all;
 
   auto load_stage = [&](int stage, int kb) {
-    const int k0 = kb * kBK;
-    for (int c = tid; c < kBM * (kBK / 8); c += kThreads) {
+    const int k0 = (kb0 + kb) * kBK;
+    for (int c = tid; c < kMmaBM * (kBK / 8); c += kMmaThreads) {
       int r = c >> 3, cc = c & 7, gr = t0 + r, gk = k0 + cc * 8;
       bool ok = gr < T && gk < d;
       const __nv_bfloat16 *src = x + (size_t)(ok ? gr : 0) * d + (ok ? gk : 0);
-      cp_async16(sX + (stage * kBM + r) * kLDS + cc * 8, src, ok);
+      cp_async16(sX + (stage * kMmaBM + r) * kLDS + cc * 8, src, ok);
     }
-    for (int c = tid; c < EP * (kBK / 8); c += kThreads) {
+    for (int c = tid; c < EP * (kBK / 8); c += kMmaThreads) {
       int r = c >> 3, cc = c & 7, gk = k0 + cc * 8;
       bool ok = r < E && gk < d;
       const __nv_bfloat16 *src = Wr + (size_t)(ok ? r : 0) * d + (ok ? gk : 0);
@@ -149,7 +160,7 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
   };
 
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
+  for (int s = 0; s < kMmaStages - 1; ++s) {
     if (s < nk) load_stage(s, s);
     cp_async_commit();
   }
@@ -161,15 +172,15 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
 
   for (int kb = 0; kb < nk; ++kb) {
-    cp_async_wait<kStages - 2>();
+    cp_async_wait<kMmaStages - 2>();
     __syncthreads();
     {
-      int nkb = kb + kStages - 1;
-      if (nkb < nk) load_stage(nkb % kStages, nkb);
+      int nkb = kb + kMmaStages - 1;
+      if (nkb < nk) load_stage(nkb % kMmaStages, nkb);
       cp_async_commit();
     }
-    const int st = kb % kStages;
-    const __nv_bfloat16 *tX = sX + (st * kBM + warp * 16) * kLDS;
+    const int st = kb % kMmaStages;
+    const __nv_bfloat16 *tX = sX + (st * kMmaBM + warp * 16) * kLDS;
     const __nv_bfloat16 *tW = sW + st * EP * kLDS;
 #pragma unroll
     for (int kk = 0; kk < kBK / 16; ++kk) {
@@ -198,7 +209,70 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     }
   }
   __syncthreads();
+  if (PARTIAL) {
+    float *part = logits + (size_t)blockIdx.y * T * E;
+    for (int i = tid; i < kMmaBM * E; i += kMmaThreads) {
+      const int r = i / E, e = i - r * E;
+      if (t0 + r < T) part[(size_t)(t0 + r) * E + e] = sZ[r * (EP + 1) + e];
+    }
+    return;
+  }
 
+  if (EP <= 32) {
+    // E <= 32: one thread per token finishes softmax and top-k serially
+    // (no shuffle chains); ties go to the lower expert id.
+    const int r = tid, s = t0 + r;
+    if (r < kMmaBM && s < T) {
+      float z[EP];
+      float m = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        float zz = -INFINITY;
+        if (e < E) {
+          zz = sZ[r * (EP + 1) + e];
+          if (bias) zz += bias[e];
+          if (zprev) zz += zscale * zprev[(size_t)s * E + e];
+          logits[(size_t)s * E + e] = zz;
+          m = fmaxf(m, zz);
+        }
+        z[e] = zz;
+      }
+      float A[EP];
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        A[e] = e < E ? expf(z[e] - m) : 0.f;
+        sum += A[e];
+      }
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        A[e] = A[e] / sum;
+        if (e < E) probs[(size_t)s * E + e] = A[e];
+      }
+      if (k > 0) {
+        uint32_t taken = 0;
+        float wsum = 0.f;
+        for (int j = 0; j < k; ++j) {
+          float bv = -INFINITY;
+          int bi = 0x7fffffff;
+#pragma unroll
+          for (int e = 0; e < EP; ++e)
+            if (e < E && !((taken >> e) & 1u) && better(z[e], e, bv, bi)) { bv = z[e]; bi = e; }
+          taken |= 1u << bi;
+          float a = 0.f;
+#pragma unroll
+          for (int e = 0; e < EP; ++e)
+            if (e == bi) a = A[e];
+          idx[(size_t)s * k + j] = bi;
+          w[(size_t)s * k + j] = a;
+          wsum += a;
+        }
+        if (renorm)
+          for (int j = 0; j < k; ++j) w[(size_t)s * k + j] = w[(size_t)s * k + j] / wsum;
+      }
+    }
+    return;
+  }
   for (int i = 0; i < 16; ++i) {
     const int r = warp * 16 + i, s = t0 + r;
     if (s >= T) break;
@@ -276,7 +350,8 @@ router_rowwise_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloa
                            const float *__restrict__ bias, const float *__restrict__ zprev,
                            float zscale, int T, int d, int E, float *__restrict__ logits,
                            float *__restrict__ probs, int k, int renorm,
-                           int32_t *__restrict__ idx, float *__restrict__ w) {
+                           int32_t *__restrict__ idx, float *__restrict__ w,
+                           unsigned long long *__restrict__ votes, int k_vote) {
   __shared__ float zs[32 * VPL];
   const int s = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int kWarps = kRowThreads / 32;
@@ -335,6 +410,86 @@ router_rowwise_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloa
     if (e < E) probs[(size_t)s * E + e] = A[v];
   }
   if (k > 0) row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
+  if (votes) {
+    // DES-Vote (i)+(ii) for this token: its top-K by P, ties to the lower
+    // id; each kept expert's vote q(P) is added to the block's total.
+    bool taken[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) taken[v] = false;
+    for (int r = 0; r < k_vote; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        if (e < E && !taken[v] && better(A[v], e, bv, bi)) { bv = A[v]; bi = e; }
+      }
+      warp_argmax(bv, bi);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v)
+        if (lane + 32 * v == bi) {
+          taken[v] = true;
+          atomicAdd(votes + bi, (unsigned long long)vote_quantum(A[v]));
+        }
+    }
+  }
+}
+
+// Finish of the split router: warp per token sums the width slices' partial
+// logits in slice order (deterministic), adds bias and gate residual, then
+// softmax, token-choice top-k and/or the DES vote (as in the rowwise kernel).
+template <int VPL>
+__global__ void __launch_bounds__(kThreads)
+router_finish_kernel(const float *__restrict__ part, int n_part, const float *__restrict__ bias,
+                     const float *__restrict__ zprev, float zscale, int T, int E,
+                     float *__restrict__ logits, float *__restrict__ probs, int k, int renorm,
+                     int32_t *__restrict__ idx, float *__restrict__ w,
+                     unsigned long long *__restrict__ votes, int k_vote) {
+  const int lane = threadIdx.x & 31;
+  const int s = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (s >= T) return;
+  float z[VPL], A[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int e = lane + 32 * v;
+    float zz = -INFINITY;
+    if (e < E) {
+      zz = 0.f;
+      for (int j = 0; j < n_part; ++j) zz += part[((size_t)j * T + s) * E + e];
+      if (bias) zz += bias[e];
+      if (zprev) zz += zscale * zprev[(size_t)s * E + e];
+      logits[(size_t)s * E + e] = zz;
+    }
+    z[v] = zz;
+  }
+  row_softmax<VPL>(z, E, A);
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int e = lane + 32 * v;
+    if (e < E) probs[(size_t)s * E + e] = A[v];
+  }
+  if (k > 0) row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
+  if (votes) {
+    bool taken[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) taken[v] = false;
+    for (int r = 0; r < k_vote; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        if (e < E && !taken[v] && better(A[v], e, bv, bi)) { bv = A[v]; bi = e; }
+      }
+      warp_argmax(bv, bi);
+#pragma unroll
+      for (int v = 0; v < VPL; ++v)
+        if (lane + 32 * v == bi) {
+          taken[v] = true;
+          atomicAdd(votes + bi, (unsigned long long)vote_quantum(A[v]));
+        }
+    }
+  }
 }
 
 template <int VPL>
@@ -361,14 +516,38 @@ int run_router_bf16(const void *x, const void *Wr, const float *bias, const floa
                     float zscale, int T, int d, int E, float *logits, float *probs, int k,
                     int renorm, int32_t *idx, float *w, cudaStream_t stream) {
   constexpr int EP = NT * 8;
-  const size_t smem = (size_t)kStages * (kBM + EP) * kLDS * sizeof(__nv_bfloat16) +
-                      (size_t)kBM * (EP + 1) * sizeof(float);
+  const size_t smem = (size_t)kMmaStages * (kMmaBM + EP) * kLDS * sizeof(__nv_bfloat16) +
+                      (size_t)kMmaBM * (EP + 1) * sizeof(float);
   auto kern = router_bf16_kernel<NT>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  dim3 grid((T + kBM - 1) / kBM);
-  kern<<<grid, kThreads, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x),
+  dim3 grid((T + kMmaBM - 1) / kMmaBM);
+  kern<<<grid, kMmaThreads, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x),
                                          static_cast<const __nv_bfloat16 *>(Wr), bias, zprev,
                                          zscale, T, d, E, logits, probs, k, renorm, idx, w);
+  return last_launch_status();
+}
+
+template <int NT>
+int run_router_split(const void *x, const void *Wr, const float *bias, const float *zprev,
+                     float zscale, int T, int d, int E, float *part, int n_part, float *logits,
+                     float *probs, int k, int renorm, int32_t *idx, float *w,
+                     unsigned long long *votes, int k_vote, cudaStream_t stream) {
+  constexpr int EP = NT * 8;
+  const size_t smem = (size_t)kMmaStages * (kMmaBM + EP) * kLDS * sizeof(__nv_bfloat16) +
+                      (size_t)kMmaBM * (EP + 1) * sizeof(float);
+  auto kern = router_bf16_kernel<NT, true>;
+  MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  dim3 grid((T + kMmaBM - 1) / kMmaBM, n_part);
+  kern<<<grid, kMmaThreads, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x),
+                                            static_cast<const __nv_bfloat16 *>(Wr), nullptr, nullptr,
+                                            0.f, T, d, E, part, nullptr, 0, 0, nullptr, nullptr);
+  MOE_CUDA_TRY(cudaPeekAtLastError());
+  const int wpb = kThreads / 32;
+  const int blocks = (T + wpb - 1) / wpb;
+  const int vpl = (E + 31) / 32;
+  if (vpl == 1) router_finish_kernel<1><<<blocks, kThreads, 0, stream>>>(part, n_part, bias, zprev, zscale, T, E, logits, probs, k, renorm, idx, w, votes, k_vote);
+  else if (vpl == 2) router_finish_kernel<2><<<blocks, kThreads, 0, stream>>>(part, n_part, bias, zprev, zscale, T, E, logits, probs, k, renorm, idx, w, votes, k_vote);
+  else router_finish_kernel<4><<<blocks, kThreads, 0, stream>>>(part, n_part, bias, zprev, zscale, T, E, logits, probs, k, renorm, idx, w, votes, k_vote);
   return last_launch_status();
 }
 
@@ -381,18 +560,47 @@ int warp_grid(int rows) {
 
 }  // namespace
 
+int router_split_parts(int T, int d, int dtype) {
+  if (dtype != MOE_BF16 || T <= 0 || T > kRowwiseMaxTokens) return 0;
+  const int tiles = (T + kMmaBM - 1) / kMmaBM;
+  const int nk = (d + kBK - 1) / kBK;
+  int parts = (2 * num_sms() + tiles - 1) / tiles;
+  if (parts > nk) parts = nk;
+  if (parts > 64) parts = 64;
+  return parts < 1 ? 1 : parts;
+}
+
+int launch_router_split(const void *x, const void *W_r, const float *bias, const float *z_prev,
+                        float z_prev_scale, int T, int d, int E, float *part, int n_part,
+                        float *logits, float *probs, int k, int renorm, int32_t *idx, float *w,
+                        int64_t *votes, int k_vote, cudaStream_t stream) {
+  if (T == 0) return MOE_OK;
+  unsigned long long *vacc = reinterpret_cast<unsigned long long *>(votes);
+  const int nt = (E + 7) / 8;
+  if (nt <= 1) return run_router_split<1>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
+  if (nt <= 2) return run_router_split<2>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
+  if (nt <= 3) return run_router_split<3>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
+  if (nt <= 4) return run_router_split<4>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
+  if (nt <= 8) return run_router_split<8>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
+  return run_router_split<16>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
+}
+
+bool router_can_vote(int T, int dtype) { return dtype == MOE_BF16 && T > 0 && T <= kRowwiseMaxTokens; }
+
 int launch_router(const void *x, const void *W_r, const float *bias, const float *z_prev,
                   float z_prev_scale, int T, int d, int E, int dtype, float *logits,
                   float *probs, int k, int renorm, int32_t *idx, float *w,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, int64_t *votes, int k_vote) {
+  if (votes && !router_can_vote(T, dtype)) return MOE_ERR_UNSUPPORTED;
+  unsigned long long *vacc = reinterpret_cast<unsigned long long *>(votes);
   if (T == 0) return MOE_OK;
   if (dtype == MOE_BF16 && T <= kRowwiseMaxTokens) {
     const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
     const __nv_bfloat16 *wb = static_cast<const __nv_bfloat16 *>(W_r);
     const int vpl = (E + 31) / 32;
-    if (vpl == 1) router_rowwise_bf16_kernel<1><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
-    else if (vpl == 2) router_rowwise_bf16_kernel<2><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
-    else router_rowwise_bf16_kernel<4><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w);
+    if (vpl == 1) router_rowwise_bf16_kernel<1><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, vacc, k_vote);
+    else if (vpl == 2) router_rowwise_bf16_kernel<2><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, vacc, k_vote);
+    else router_rowwise_bf16_kernel<4><<<T, kRowThreads, 0, stream>>>(xb, wb, bias, z_prev, z_prev_scale, T, d, E, logits, probs, k, renorm, idx, w, vacc, k_vote);
     return last_launch_status();
   }
   if (dtype == MOE_BF16) {

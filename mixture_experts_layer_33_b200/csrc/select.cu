@@ -125,11 +125,6 @@ expert_choice_kernel(const float *__restrict__ probs, int E, int S, int C,
 
 constexpr int kDesThreads = 1024;  // one warp per token of a 32-token block
 
-// q(p) = round-half-even(p * 2^40): exact in double, then rounded once.
-__device__ __forceinline__ long long vote_quantum(float p) {
-  return __double2ll_rn((double)p * 1099511627776.0);
-}
-
 // One CTA for the whole block of N tokens; each lane holds kDesVpl of a
 // token's M <= 32*kDesVpl probabilities.
 template <int kDesVpl>
@@ -226,6 +221,65 @@ des_vote_kernel(const float *__restrict__ P, int N, int M, int K, int Mc,
   }
 }
 
+// Small-block DES tail, parallel over tokens: the votes were summed into
+// `votes` (exact int64, order-free) by the router's per-token CTAs; every
+// CTA here re-derives the same election from them (M <= 256 values) and
+// re-routes its own token over the core set. CTA 0 also writes the core set.
+template <int VPL>
+__global__ void __launch_bounds__(256)
+des_reroute_kernel(const float *__restrict__ P, const int64_t *__restrict__ votes, int N, int M,
+                   int K, int Mc, int32_t *__restrict__ core, int32_t *__restrict__ idx,
+                   float *__restrict__ w) {
+  __shared__ int in_core[MOE_MAX_EXPERTS];
+  const int n = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < M; e += blockDim.x) {
+    const long long ve = votes[e];
+    int rank = 0;
+    for (int f = 0; f < M; ++f) {
+      const long long vf = votes[f];
+      rank += (vf > ve) || (vf == ve && f < e);
+    }
+    in_core[e] = rank < Mc;
+  }
+  __syncthreads();
+  if (n == 0)
+    for (int e = tid; e < M; e += blockDim.x)
+      if (in_core[e]) {
+        int pos = 0;
+        for (int f = 0; f < e; ++f) pos += in_core[f];
+        core[pos] = e;
+      }
+  if (warp != 0) return;
+  float p[VPL];
+  bool taken[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int e = lane + 32 * v;
+    const bool ok = e < M && in_core[e];
+    p[v] = ok ? P[(size_t)n * M + e] : -INFINITY;
+    taken[v] = !ok;
+  }
+  for (int r = 0; r < K; ++r) {
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int e = lane + 32 * v;
+      if (!taken[v] && better(p[v], e, bv, bi)) { bv = p[v]; bi = e; }
+    }
+    warp_argmax(bv, bi);
+    float own = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+      if (lane + 32 * v == bi) { taken[v] = true; own = p[v]; }
+    const float pw = __shfl_sync(0xffffffffu, own, bi & 31);
+    if (lane == 0) {
+      idx[(size_t)n * K + r] = bi;
+      w[(size_t)n * K + r] = pw;
+    }
+  }
+}
+
 }  // namespace
 
 int launch_expert_choice(const float *probs, int T, int E, int S, int C, int32_t *tok,
@@ -237,6 +291,16 @@ int launch_expert_choice(const float *probs, int T, int E, int S, int C, int32_t
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   int threads = S < kEcThreads ? ((S + 31) / 32) * 32 : kEcThreads;
   expert_choice_kernel<<<G * E, threads, smem, stream>>>(probs, E, S, C, tok, w);
+  return last_launch_status();
+}
+
+int launch_des_reroute(const float *probs, const int64_t *votes, int N, int M, int K, int M_core,
+                       int32_t *core, int32_t *idx, float *w, cudaStream_t stream) {
+  if (N == 0) return MOE_OK;
+  if (M <= 32) des_reroute_kernel<1><<<N, 256, 0, stream>>>(probs, votes, N, M, K, M_core, core, idx, w);
+  else if (M <= 64) des_reroute_kernel<2><<<N, 256, 0, stream>>>(probs, votes, N, M, K, M_core, core, idx, w);
+  else if (M <= 128) des_reroute_kernel<4><<<N, 256, 0, stream>>>(probs, votes, N, M, K, M_core, core, idx, w);
+  else des_reroute_kernel<8><<<N, 256, 0, stream>>>(probs, votes, N, M, K, M_core, core, idx, w);
   return last_launch_status();
 }
 

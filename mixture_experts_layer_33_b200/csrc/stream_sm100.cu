@@ -20,7 +20,7 @@
 //   warp 0      TMA producer: a ring of 40 KB stages [A0 | A1 | B0 | B1]
 //               (two 128x64 weight tiles, two NBx64 token tiles)
 //   warp 1      one thread issues tcgen05.mma, 8 per stage
-//   warps 2..5  epilogue, one TMEM lane quadrant each
+//   warps 2..5  epilogue, one TMEM lane quadrant each (outputs in bf16)
 // Stage use: SwiGLU up: A0 = gate rows, A1 = up rows, both against B0, into
 // two accumulators, so the same thread forms silu(gate) * up. GELU up and
 // down: A0/B0 and A1/B1 are two consecutive 64-wide k-blocks of one
@@ -331,8 +331,7 @@ expert_stream_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
           for (int i = 0; i < 32; ++i) {
             if (c + i < cnt) {
               const int64_t o = (int64_t)(row0 + c + i) * pd.ld_out + feat;
-              if (up) static_cast<__nv_bfloat16 *>(pd.out)[o] = __float2bfloat16_rn(v[i]);
-              else static_cast<float *>(pd.out)[o] = v[i];
+              static_cast<__nv_bfloat16 *>(pd.out)[o] = __float2bfloat16_rn(v[i]);
             }
           }
         }

@@ -124,11 +124,14 @@ def test_independent_routing_flips_are_near_ties(name):
         assert abs(kth_ref - gpu_min) <= 1e-5 * scale
 
 
-@pytest.mark.parametrize("name,over", SMALL[1:4], ids=[s[0] for s in SMALL[1:4]])
+STAGEWISE = SMALL[1:5] + [("ditmoe_xl_2sm", PAIR[0][1])]
+
+
+@pytest.mark.parametrize("name,over", STAGEWISE, ids=[s[0] for s in STAGEWISE])
 def test_stagewise_entry_points(name, over):
     """Each entry point alone: router -> select -> dispatch -> grouped MLP -> combine."""
     m = H.moe()
-    cfg = gen.workload(name, **over)
+    cfg = gen.workload(name.replace("_2sm", ""), **over)
     inp = gen.make_inputs(cfg, "cuda")
     hin = H.host(inp)
     c = m.make_config(cfg)
@@ -180,12 +183,12 @@ def test_stagewise_entry_points(name, over):
         np.testing.assert_array_equal(tok_assign.cpu().numpy(), o_tass)
     assert torch.equal(x_perm[:n_rows], inp["x"][perm[:n_rows].long()])
 
-    y_perm = torch.empty(na, d, device=dev)
-    y_sh = torch.empty(T, d, device=dev) if cfg["n_shared"] else None
+    y_perm = torch.empty(na, d, dtype=inp["x"].dtype, device=dev)
+    y_sh = torch.empty(T, d, dtype=inp["x"].dtype, device=dev) if cfg["n_shared"] else None
     m.grouped_mlp(c, x_perm, offsets, inp["W1"], inp["W2"], inp["x"], inp["Ws1"], inp["Ws2"],
                   y_perm, y_sh, status, ws)
     torch.cuda.synchronize()
-    yp = y_perm.cpu().numpy()[:n_rows]
+    yp = gen.to_numpy_f32(y_perm)[:n_rows]
     ref_rows = np.empty_like(yp, dtype=np.float64)
     for e in range(cfg["E_heavy"]):
         lo, hi = o_off[e], o_off[e + 1]
@@ -195,7 +198,7 @@ def test_stagewise_entry_points(name, over):
     assert H.normwise(yp, ref_rows) <= H.Y_TOL[cfg["dtype"]]
     if y_sh is not None:
         ref_sh = oracle.mlp_gelu(hin["x"], hin["Ws1"], hin["Ws2"])
-        assert H.normwise(y_sh.cpu().numpy(), ref_sh) <= H.Y_TOL[cfg["dtype"]]
+        assert H.normwise(gen.to_numpy_f32(y_sh), ref_sh) <= H.Y_TOL[cfg["dtype"]]
 
     y = torch.empty_like(inp["x"])
     m.combine(c, y_perm, y_sh, sel, w, row_of, tok_ptr, tok_assign, inp["x"],
