@@ -53,16 +53,18 @@ class L2Flush:
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the grouped-MLP
 # launches of one layer pass, from one ncu capture (profiles/), valid only while
-# the GEMM kernel source is byte-identical to the one profiled.
+# the profiled kernel source is byte-identical to the one captured.
 NCU_TRAFFIC = {
-    "ditmoe_xl": {"bytes": (163.87 + 252.31 + 500.84 + 97.23) * 1e6,
-                  "gemm_source_sha256_16": "b9d44b6780bae36a"},
+    "ditmoe_xl": {"bytes": (162.94 + 259.05 + 513.45 + 48.33) * 1e6,
+                  "source": "gemm_sm100.cu", "sha256_16": "e8ddefae01ad9317"},
+    "des_vote": {"bytes": (404.05 + 4.51) * 1e6,
+                 "source": "stream_sm100.cu", "sha256_16": "71f52938b36fd91f"},
 }
 
 
-def gemm_source_hash():
+def source_hash(name):
     import hashlib
-    path = os.path.join(ROOT, "mixture_experts_layer_33_b200", "csrc", "gemm_sm100.cu")
+    path = os.path.join(ROOT, "mixture_experts_layer_33_b200", "csrc", name)
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
@@ -425,12 +427,15 @@ def gpu_bench(args):
 
     peaks, peak_src = load_peaks()
     tr = NCU_TRAFFIC.get(cfg["name"])
-    traffic = tr["bytes"] if tr and tr["gemm_source_sha256_16"] == gemm_source_hash() else None
+    traffic = tr["bytes"] if tr and tr["sha256_16"] == source_hash(tr["source"]) else None
     gm_ms = stage_ms["grouped_mlp"] / args.steps  # grouped-MLP launches, from timed region 2
     if cfg["routing"] == "des_vote":
         bytes_ = weight_bytes_used(cfg, used)
         achieved = bytes_ / (gm_ms / 1e3) / 1e9
-        roof = {"bound": "hbm", "kernel": "grouped_mlp (GEMM1 + GEMM2 launches)",
+        kname = ("expert_stream_kernel (weight-streaming expert MLP, one launch)"
+                 if cfg["T"] <= 128 and cfg["dtype"] == "bf16"
+                 else "grouped_mlp (GEMM1 + GEMM2 launches)")
+        roof = {"bound": "hbm", "kernel": kname,
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "algorithmic_per_launch": bytes_, "peak_source": peak_src}
