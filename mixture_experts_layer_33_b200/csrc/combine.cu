@@ -11,10 +11,13 @@
 //
 // One warp per (token, 256-feature chunk); each lane owns 8 consecutive
 // features and reads them with 16-byte loads; a token's slot metadata is
-// loaded once, one slot per lane, and broadcast by shuffles. Expert outputs
-// arrive in the layer dtype; the sum runs in fp32 in slot order (no atomics,
-// so the output is bitwise deterministic) and is rounded once. `residual`
-// may alias `y` (the forward pass writes x + shared(x) into y first).
+// loaded once, one slot per lane, turned into a source row per slot and
+// broadcast by shuffles; the rows of four slots are loaded before any is
+// summed, so a token's loads overlap instead of queueing one behind the
+// other. Expert outputs arrive in the layer dtype; the sum runs in fp32 in
+// slot order (no atomics, so the output is bitwise deterministic) and is
+// rounded once. `residual` may alias `y` (the forward pass writes
+// x + shared(x) into y first).
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,6 +25,36 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kBatch = 4;  // slots whose rows are in flight together
+
+// 8 consecutive elements held raw until they are summed.
+template <typename T> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16 *p) { u = *reinterpret_cast<const uint4 *>(p); }
+  __device__ __forceinline__ void fma_into(float wgt, float (&acc)[8]) const {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      acc[2 * i] = fmaf(wgt, f.x, acc[2 * i]);
+      acc[2 * i + 1] = fmaf(wgt, f.y, acc[2 * i + 1]);
+    }
+  }
+};
+template <> struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float *p) {
+    a = *reinterpret_cast<const float4 *>(p);
+    b = *reinterpret_cast<const float4 *>(p + 4);
+  }
+  __device__ __forceinline__ void fma_into(float wgt, float (&acc)[8]) const {
+    acc[0] = fmaf(wgt, a.x, acc[0]); acc[1] = fmaf(wgt, a.y, acc[1]);
+    acc[2] = fmaf(wgt, a.z, acc[2]); acc[3] = fmaf(wgt, a.w, acc[3]);
+    acc[4] = fmaf(wgt, b.x, acc[4]); acc[5] = fmaf(wgt, b.y, acc[5]);
+    acc[6] = fmaf(wgt, b.z, acc[6]); acc[7] = fmaf(wgt, b.w, acc[7]);
+  }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTable kinds) {
@@ -56,40 +89,46 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
       for (int i = 0; i < 8; ++i) acc[i] += t[i];
     }
     for (int j0 = a0; j0 < a1; j0 += 32) {
-      // Lane j holds the metadata of slot j0 + j; the slot loop broadcasts it.
-      int m_kind = MOE_ZERO, m_row = -1, m_ci = 0;
+      // Lane j holds slot j0 + j: its weight and the first element of its
+      // source row (the expert's output row, x for an identity expert, the
+      // learned vector for a constant expert), or none (zero expert, a row
+      // the dispatch dropped, or an id it flagged).
+      const T *m_src = nullptr;
       float m_w = 0.f;
       if (j0 + lane < a1) {
         const int asg = ec ? a.tok_assign[j0 + lane] : j0 + lane;
         const int e = ec ? (int)((asg / a.C) % a.E) : a.sel[asg];
-        if (e >= 0 && e < a.E) {  // out-of-range ids were flagged by dispatch
-          m_kind = kinds.kind[e];
-          m_w = a.w[asg];
-          m_row = m_kind == MOE_HEAVY ? a.row_of[asg] : -1;
-          m_ci = kinds.cidx[e];
+        const int row = a.row_of[asg];
+        const float wv = a.w[asg];
+        if (e >= 0 && e < a.E) {
+          const int kind = kinds.kind[e];
+          if (kind == MOE_HEAVY) {
+            if (row >= 0) m_src = yp + (size_t)row * a.d;
+          } else if (kind == MOE_IDENTITY) {
+            m_src = x + (size_t)s * a.d;
+          } else if (kind == MOE_CONST) {
+            m_src = cv + (size_t)kinds.cidx[e] * a.d;
+          }
+          m_w = wv;
         }
       }
       const int nj = min(32, a1 - j0);
-#pragma unroll 2
-      for (int j = 0; j < nj; ++j) {
-        const int kind = __shfl_sync(0xffffffffu, m_kind, j);
-        const float wgt = __shfl_sync(0xffffffffu, m_w, j);
-        const int row = __shfl_sync(0xffffffffu, m_row, j);
-        const int ci = __shfl_sync(0xffffffffu, m_ci, j);
-        if (!live) continue;
-        float t[8];
-        if (kind == MOE_HEAVY) {
-          if (row < 0) continue;
-          load8(yp + (size_t)row * a.d + c0, t);
-        } else if (kind == MOE_IDENTITY) {
-          load8(x + (size_t)s * a.d + c0, t);
-        } else if (kind == MOE_CONST) {
-          load8(cv + (size_t)ci * a.d + c0, t);
-        } else {
-          continue;  // zero expert: contributes nothing
+      for (int jb = 0; jb < nj; jb += kBatch) {
+        Raw8<T> raw[kBatch];
+        const T *src[kBatch];
+        float wgt[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          const int j = (jb + u) & 31;
+          src[u] = reinterpret_cast<const T *>(
+              __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(m_src), j));
+          wgt[u] = __shfl_sync(0xffffffffu, m_w, j);
+          if (jb + u >= nj || !live) src[u] = nullptr;
+          if (src[u]) raw[u].load(src[u] + c0);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wgt, t[i], acc[i]);
+        for (int u = 0; u < kBatch; ++u)
+          if (src[u]) raw[u].fma_into(wgt[u], acc);
       }
     }
     if (live) store8(y + (size_t)s * a.d + c0, acc);

@@ -43,6 +43,45 @@ int launch_router_split(const void *x, const void *W_r, const float *bias, const
                         float z_prev_scale, int T, int d, int E, float *part, int n_part,
                         float *logits, float *probs, int k, int renorm, int32_t *idx, float *w,
                         int64_t *votes, int k_vote, cudaStream_t stream);
+// Words zeroed by the first CTA of the split router, for kernels later in
+// the same stream (DES vote totals, a grid-barrier counter, counters).
+struct ZeroList {
+  int32_t *p[3];
+  int n[3];
+};
+int launch_router_partial(const void *x, const void *W_r, int T, int d, int E, float *part,
+                          int n_part, const ZeroList &zero, cudaStream_t stream);
+
+// small_route.cu: router finish + DES election/re-route + dispatch + row
+// gather for blocks of at most 128 tokens, one cooperative launch (one CTA
+// per token, bounded grid barriers). Reads the split router's partials.
+constexpr int kSmallRouteMaxTokens = 128;
+constexpr int kSmallRouteMaxK = 32;
+constexpr int kSmallRouteMaxAssign = 2048;
+struct SmallRouteArgs {
+  const float *part;     // [n_part][T][E] partial logits
+  int n_part;
+  const float *bias, *zprev;
+  float zscale;
+  int T, E, n_heavy, k, routing, renorm, M_core;
+  int row_vecs;          // 16-byte vectors per x row
+  const uint4 *x;        // [T][row_vecs]
+  uint4 *x_perm;         // [rows][row_vecs]
+  float *logits, *probs; // [T][E]
+  int32_t *sel;          // [T*k] expert per slot
+  float *w;              // [T*k] routing weight per slot
+  unsigned long long *votes;  // [E] zeroed before the launch (DES)
+  int32_t *core;         // [M_core] (DES)
+  int32_t *offsets;      // [n_heavy + 1]
+  int32_t *perm;         // [rows] token of each expert row
+  int32_t *row_of;       // [T*k] expert row of each slot, -1 if none
+  unsigned *barrier;     // grid-barrier counter, zeroed before the launch
+  unsigned *gmask;       // [n_heavy][4] token bitmasks, zeroed before the launch
+  int32_t *dev_status;
+};
+bool small_route_supported(int T, int E, int k, int routing, int dtype);
+int launch_small_route(const SmallRouteArgs &args, cudaStream_t stream);
+
 int launch_select_topk(const float *logits, const float *probs, int T, int E,
                        int k, int renorm, int32_t *idx, float *w,
                        cudaStream_t stream);

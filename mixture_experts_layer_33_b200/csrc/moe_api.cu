@@ -82,7 +82,7 @@ int n_const_of(const moe_config &c) {
 // Workspace layout shared by the entry points.
 struct Layout {
   size_t logits, probs, sel, w, votes, core, offsets, perm, row_of, tok_ptr, tok_assign, dpart,
-      x_perm, H, H_sh, Y, Y_sh, done, rpart, x_dev, res_dev, zp_dev, y_dev, total;
+      x_perm, H, H_sh, Y, Y_sh, done, rpart, cbar, x_dev, res_dev, zp_dev, y_dev, total;
 };
 
 Layout layout_of(const moe_config &c) {
@@ -112,6 +112,9 @@ Layout layout_of(const moe_config &c) {
   L.Y_sh = take(hs ? (size_t)c.T * c.d * eb : 0);
   L.done = take(stream_mlp_workspace_bytes(c.n_heavy + 1));  // routed groups, then the shared one
   L.rpart = take((size_t)router_split_parts(c.T, c.d, c.dtype) * c.T * c.E * 4);
+  // Small-block routing kernel: grid-barrier counter (16 B), then a 4-word
+  // token bitmask per expert.
+  L.cbar = take(16 + (size_t)c.E * 16);
   L.x_dev = take((size_t)c.T * c.d * eb);
   L.res_dev = take((size_t)c.T * c.d * eb);
   L.zp_dev = take((size_t)c.T * c.E * 4);
@@ -250,12 +253,43 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
 
   int st = MOE_OK;
   const int n_part = router_split_parts(c.T, c.d, c.dtype);
-  if (n_part > 0 && c.routing != MOE_EXPERT_CHOICE) {
+  const bool streaming = c.dtype == MOE_BF16 && stream_mlp_supported(c.T);
+  bool routed_and_gathered = false;
+  if (n_part > 0 && small_route_supported(c.T, c.E, c.k, c.routing, c.dtype)) {
+    // Small bf16 block (<= 128 tokens): the router split over the model
+    // width, then one cooperative kernel finishes the router, selects (DES:
+    // votes, elects, re-routes), dispatches and gathers the rows. The split
+    // router clears the vote totals, the barrier counter and the
+    // weight-streaming kernel's counters on its way.
+    const bool des = c.routing == MOE_DES_VOTE;
+    ZeroList zero{};
+    zero.p[0] = at<int32_t>(ws, L.cbar);
+    zero.n[0] = 4 + 4 * c.E;
+    if (des) { zero.p[1] = reinterpret_cast<int32_t *>(votes); zero.n[1] = 2 * c.E; }
+    if (streaming) { zero.p[2] = at<int32_t>(ws, L.done); zero.n[2] = c.n_heavy + 1; }
+    st = launch_router_partial(x, W_r, c.T, c.d, c.E, at<float>(ws, L.rpart), n_part, zero, stream);
+    if (st != MOE_OK) return st;
+    SmallRouteArgs sa{};
+    sa.part = at<float>(ws, L.rpart); sa.n_part = n_part;
+    sa.bias = bias; sa.zprev = z_prev; sa.zscale = c.gate_residual_scale;
+    sa.T = c.T; sa.E = c.E; sa.n_heavy = c.n_heavy; sa.k = c.k; sa.routing = c.routing;
+    sa.renorm = c.renorm; sa.M_core = c.M_core;
+    sa.row_vecs = (int)((int64_t)c.d * elem_bytes(c.dtype) / 16);
+    sa.x = static_cast<const uint4 *>(x); sa.x_perm = static_cast<uint4 *>(x_perm);
+    sa.logits = logits; sa.probs = probs; sa.sel = sel; sa.w = w;
+    sa.votes = reinterpret_cast<unsigned long long *>(votes); sa.core = core;
+    sa.offsets = offsets; sa.perm = perm; sa.row_of = row_of;
+    sa.barrier = at<unsigned>(ws, L.cbar); sa.gmask = at<unsigned>(ws, L.cbar) + 4;
+    sa.dev_status = dev_status;
+    st = launch_small_route(sa, stream);
+    if (st != MOE_OK) return st;
+    routed_and_gathered = true;
+  } else if (n_part > 0 && c.routing != MOE_EXPERT_CHOICE) {
     // Small bf16 block: router split over the model width, then a per-token
     // finish that also selects (token choice) or sums the exact int64 DES
-    // votes; DES then elects the core set and re-routes per token.
+    // votes (cleared by the split router); DES then elects the core set and
+    // re-routes per token.
     const bool des = c.routing == MOE_DES_VOTE;
-    if (des) MOE_CUDA_TRY(cudaMemsetAsync(votes, 0, (size_t)c.E * sizeof(int64_t), stream));
     st = launch_router_split(x, W_r, bias, z_prev, c.gate_residual_scale, c.T, c.d, c.E,
                              at<float>(ws, L.rpart), n_part, logits, probs, des ? 0 : c.k,
                              c.renorm, des ? nullptr : sel, des ? nullptr : w,
@@ -273,17 +307,18 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
       st = launch_des_vote(probs, c.T, c.E, c.k, c.M_core, votes, core, sel, w, stream);
     if (st != MOE_OK) return st;
   }
-  DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
-  const bool streaming = c.dtype == MOE_BF16 && stream_mlp_supported(c.T);
-  if (streaming) {  // the dispatch clears the weight-streaming kernel's counters
-    da.zero_words = at<int32_t>(ws, L.done);
-    da.n_zero_words = c.n_heavy + 1;
-  }
-  st = launch_dispatch(da, at<void>(ws, L.dpart), stream);
-  if (st != MOE_OK) return st;
-  if (c.n_heavy > 0) {
-    st = launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, na, c.d, elem_bytes(c.dtype), stream);
+  if (!routed_and_gathered) {
+    DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
+    if (streaming) {  // the dispatch clears the weight-streaming kernel's counters
+      da.zero_words = at<int32_t>(ws, L.done);
+      da.n_zero_words = c.n_heavy + 1;
+    }
+    st = launch_dispatch(da, at<void>(ws, L.dpart), stream);
     if (st != MOE_OK) return st;
+    if (c.n_heavy > 0) {
+      st = launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, na, c.d, elem_bytes(c.dtype), stream);
+      if (st != MOE_OK) return st;
+    }
   }
   // bf16 grouped-GEMM path with a shared expert: its down-projection epilogue
   // writes y = residual + shared(x) straight into y, and the combine then adds

@@ -29,10 +29,8 @@
 namespace moe {
 namespace {
 
-constexpr int kBM = 64;        // tokens per CTA
 constexpr int kBK = 64;        // model-width slice per pipeline stage
 constexpr int kLDS = kBK + 8;  // padded smem row (bf16): conflict-free ldmatrix
-constexpr int kStages = 3;
 constexpr int kThreads = 128;
 constexpr int kRowwiseMaxTokens = 512;  // bf16 layers this small use one CTA per token
 constexpr int kMmaBM = 32;               // tokens per CTA of the MMA router (2 warps x 16)
@@ -128,7 +126,8 @@ __global__ void __launch_bounds__(kMmaThreads)
 router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ Wr,
                    const float *__restrict__ bias, const float *__restrict__ zprev, float zscale,
                    int T, int d, int E, float *__restrict__ logits, float *__restrict__ probs,
-                   int k, int renorm, int32_t *__restrict__ idx, float *__restrict__ w) {
+                   int k, int renorm, int32_t *__restrict__ idx, float *__restrict__ w,
+                   ZeroList zero) {
   constexpr int EP = NT * 8;
   constexpr int VPL = (EP + 31) / 32;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -137,6 +136,11 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
   float *sZ = reinterpret_cast<float *>(sW + kMmaStages * EP * kLDS);    // [kMmaBM][EP + 1]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (PARTIAL && blockIdx.x == 0 && blockIdx.y == 0) {
+#pragma unroll
+    for (int l = 0; l < 3; ++l)
+      for (int i = tid; i < zero.n[l]; i += kMmaThreads) zero.p[l][i] = 0;
+  }
   const int t0 = blockIdx.x * kMmaBM;
   const int nk_all = (d + kBK - 1) / kBK;
   const int kb_per = PARTIAL ? (nk_all + gridDim.y - 1) / gridDim.y : nk_all;
@@ -218,7 +222,7 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
     return;
   }
 
-  if (EP <= 32) {
+  if constexpr (EP <= 32) {
     // E <= 32: one thread per token finishes softmax and top-k serially
     // (no shuffle chains); ties go to the lower expert id.
     const int r = tid, s = t0 + r;
@@ -271,31 +275,31 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
           for (int j = 0; j < k; ++j) w[(size_t)s * k + j] = w[(size_t)s * k + j] / wsum;
       }
     }
-    return;
-  }
-  for (int i = 0; i < 16; ++i) {
-    const int r = warp * 16 + i, s = t0 + r;
-    if (s >= T) break;
-    float z[VPL], A[VPL];
+  } else {
+    for (int i = 0; i < 16; ++i) {
+      const int r = warp * 16 + i, s = t0 + r;
+      if (s >= T) break;
+      float z[VPL], A[VPL];
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      int e = lane + 32 * v;
-      float zz = -INFINITY;
-      if (e < E) {
-        zz = sZ[r * (EP + 1) + e];
-        if (bias) zz += bias[e];
-        if (zprev) zz += zscale * zprev[(size_t)s * E + e];
-        logits[(size_t)s * E + e] = zz;
+      for (int v = 0; v < VPL; ++v) {
+        int e = lane + 32 * v;
+        float zz = -INFINITY;
+        if (e < E) {
+          zz = sZ[r * (EP + 1) + e];
+          if (bias) zz += bias[e];
+          if (zprev) zz += zscale * zprev[(size_t)s * E + e];
+          logits[(size_t)s * E + e] = zz;
+        }
+        z[v] = zz;
       }
-      z[v] = zz;
-    }
-    row_softmax<VPL>(z, E, A);
+      row_softmax<VPL>(z, E, A);
 #pragma unroll
-    for (int v = 0; v < VPL; ++v) {
-      int e = lane + 32 * v;
-      if (e < E) probs[(size_t)s * E + e] = A[v];
+      for (int v = 0; v < VPL; ++v) {
+        int e = lane + 32 * v;
+        if (e < E) probs[(size_t)s * E + e] = A[v];
+      }
+      if (k > 0) row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
     }
-    if (k > 0) row_topk<VPL>(z, A, E, k, renorm, idx + (size_t)s * k, w + (size_t)s * k);
   }
 }
 
@@ -455,6 +459,7 @@ router_finish_kernel(const float *__restrict__ part, int n_part, const float *__
     float zz = -INFINITY;
     if (e < E) {
       zz = 0.f;
+#pragma unroll 8
       for (int j = 0; j < n_part; ++j) zz += part[((size_t)j * T + s) * E + e];
       if (bias) zz += bias[e];
       if (zprev) zz += zscale * zprev[(size_t)s * E + e];
@@ -523,15 +528,13 @@ int run_router_bf16(const void *x, const void *Wr, const float *bias, const floa
   dim3 grid((T + kMmaBM - 1) / kMmaBM);
   kern<<<grid, kMmaThreads, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x),
                                          static_cast<const __nv_bfloat16 *>(Wr), bias, zprev,
-                                         zscale, T, d, E, logits, probs, k, renorm, idx, w);
+                                         zscale, T, d, E, logits, probs, k, renorm, idx, w, ZeroList{});
   return last_launch_status();
 }
 
 template <int NT>
-int run_router_split(const void *x, const void *Wr, const float *bias, const float *zprev,
-                     float zscale, int T, int d, int E, float *part, int n_part, float *logits,
-                     float *probs, int k, int renorm, int32_t *idx, float *w,
-                     unsigned long long *votes, int k_vote, cudaStream_t stream) {
+int run_router_partial(const void *x, const void *Wr, int T, int d, int E, float *part,
+                       int n_part, const ZeroList &zero, cudaStream_t stream) {
   constexpr int EP = NT * 8;
   const size_t smem = (size_t)kMmaStages * (kMmaBM + EP) * kLDS * sizeof(__nv_bfloat16) +
                       (size_t)kMmaBM * (EP + 1) * sizeof(float);
@@ -540,8 +543,23 @@ int run_router_split(const void *x, const void *Wr, const float *bias, const flo
   dim3 grid((T + kMmaBM - 1) / kMmaBM, n_part);
   kern<<<grid, kMmaThreads, smem, stream>>>(static_cast<const __nv_bfloat16 *>(x),
                                             static_cast<const __nv_bfloat16 *>(Wr), nullptr, nullptr,
-                                            0.f, T, d, E, part, nullptr, 0, 0, nullptr, nullptr);
-  MOE_CUDA_TRY(cudaPeekAtLastError());
+                                            0.f, T, d, E, part, nullptr, 0, 0, nullptr, nullptr,
+                                            zero);
+  return last_launch_status();
+}
+
+template <int NT>
+int run_router_split(const void *x, const void *Wr, const float *bias, const float *zprev,
+                     float zscale, int T, int d, int E, float *part, int n_part, float *logits,
+                     float *probs, int k, int renorm, int32_t *idx, float *w,
+                     unsigned long long *votes, int k_vote, cudaStream_t stream) {
+  ZeroList zero{};
+  if (votes) {  // the partial kernel clears the vote totals the finish adds into
+    zero.p[0] = reinterpret_cast<int32_t *>(votes);
+    zero.n[0] = 2 * E;
+  }
+  const int st = run_router_partial<NT>(x, Wr, T, d, E, part, n_part, zero, stream);
+  if (st != MOE_OK) return st;
   const int wpb = kThreads / 32;
   const int blocks = (T + wpb - 1) / wpb;
   const int vpl = (E + 31) / 32;
@@ -583,6 +601,18 @@ int launch_router_split(const void *x, const void *W_r, const float *bias, const
   if (nt <= 4) return run_router_split<4>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
   if (nt <= 8) return run_router_split<8>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
   return run_router_split<16>(x, W_r, bias, z_prev, z_prev_scale, T, d, E, part, n_part, logits, probs, k, renorm, idx, w, vacc, k_vote, stream);
+}
+
+int launch_router_partial(const void *x, const void *W_r, int T, int d, int E, float *part,
+                          int n_part, const ZeroList &zero, cudaStream_t stream) {
+  if (T == 0) return MOE_OK;
+  const int nt = (E + 7) / 8;
+  if (nt <= 1) return run_router_partial<1>(x, W_r, T, d, E, part, n_part, zero, stream);
+  if (nt <= 2) return run_router_partial<2>(x, W_r, T, d, E, part, n_part, zero, stream);
+  if (nt <= 3) return run_router_partial<3>(x, W_r, T, d, E, part, n_part, zero, stream);
+  if (nt <= 4) return run_router_partial<4>(x, W_r, T, d, E, part, n_part, zero, stream);
+  if (nt <= 8) return run_router_partial<8>(x, W_r, T, d, E, part, n_part, zero, stream);
+  return run_router_partial<16>(x, W_r, T, d, E, part, n_part, zero, stream);
 }
 
 bool router_can_vote(int T, int dtype) { return dtype == MOE_BF16 && T > 0 && T <= kRowwiseMaxTokens; }
