@@ -82,6 +82,46 @@ struct SmallRouteArgs {
 bool small_route_supported(int T, int E, int k, int routing, int dtype);
 int launch_small_route(const SmallRouteArgs &args, cudaStream_t stream);
 
+// block_sm100.cu: the whole layer for blocks of <= 128 bf16 tokens (token
+// choice or DES-Vote, no shared expert) in one persistent cooperative
+// kernel: router (K-sliced over the CTAs), selection, weight-streaming MLP
+// (up projection over all tokens, no dispatch), combine. Its sync words,
+// bitmasks, vote totals and counters sit in one workspace region that must
+// be zero at launch (block_zero_bytes).
+struct BlockArgs {
+  const void *W_r;       // [E][d] bf16 router weights
+  float *part;           // [n_slices][T][E] partial logits (workspace)
+  int n_slices, kslice;  // router K slices over the CTAs, columns per slice
+  const float *bias, *zprev;
+  float zscale;
+  int T, E, n_heavy, k, routing, renorm, M_core;
+  int d, h;              // model width, expert hidden width
+  int w1_rows_per_group; // h (GELU) or 2h (SwiGLU: gate rows, then up rows)
+  const void *x;         // [T][d] bf16
+  const void *residual;  // [T][d] bf16, may alias y
+  const void *const_vecs;
+  void *y;               // [T][d] bf16
+  void *H, *Y;           // [T*k][h], [T*k][d] bf16 workspace
+  float *logits, *probs;
+  int32_t *sel;
+  float *w;
+  int64_t *votes_out;    // DES vote totals for the caller
+  int32_t *core, *offsets, *perm, *row_of;
+  // The zeroed region (block_zero_bytes), split by block_zero_layout:
+  unsigned *sync;        // [0] barrier arrivals, [1] finished CTAs, [2] unit tickets
+  unsigned *gmask;       // [E][4] token bitmasks
+  unsigned long long *votes;  // [E] DES vote totals (exact fixed point)
+  int32_t *done;         // [n_heavy] up-unit arrivals per expert
+  int32_t *dev_status;
+};
+bool moe_block_supported(const moe_config &c);
+int block_router_slices(int d, int *kslice);  // K slices of the in-kernel router
+size_t block_zero_bytes(int E, int n_heavy);
+// Points a's sync / gmask / votes / done into the zeroed region `z`.
+void block_zero_layout(BlockArgs &a, void *z, int E);
+int launch_moe_block(const BlockArgs &a, const KindTable &kinds, const void *W1, const void *W2,
+                     int act, cudaStream_t stream);
+
 int launch_select_topk(const float *logits, const float *probs, int T, int E,
                        int k, int renorm, int32_t *idx, float *w,
                        cudaStream_t stream);

@@ -82,7 +82,7 @@ int n_const_of(const moe_config &c) {
 // Workspace layout shared by the entry points.
 struct Layout {
   size_t logits, probs, sel, w, votes, core, offsets, perm, row_of, tok_ptr, tok_assign, dpart,
-      x_perm, H, H_sh, Y, Y_sh, done, rpart, cbar, x_dev, res_dev, zp_dev, y_dev, total;
+      x_perm, H, H_sh, Y, Y_sh, done, rpart, bzero, cbar, x_dev, res_dev, zp_dev, y_dev, total;
 };
 
 Layout layout_of(const moe_config &c) {
@@ -111,7 +111,13 @@ Layout layout_of(const moe_config &c) {
   L.Y = take((size_t)na * c.d * eb);
   L.Y_sh = take(hs ? (size_t)c.T * c.d * eb : 0);
   L.done = take(stream_mlp_workspace_bytes(c.n_heavy + 1));  // routed groups, then the shared one
-  L.rpart = take((size_t)router_split_parts(c.T, c.d, c.dtype) * c.T * c.E * 4);
+  {
+    int ks = 0;
+    const int parts = router_split_parts(c.T, c.d, c.dtype);
+    const int slices = moe_block_supported(c) ? block_router_slices(c.d, &ks) : 0;
+    L.rpart = take((size_t)(parts > slices ? parts : slices) * c.T * c.E * 4);
+  }
+  L.bzero = take(moe_block_supported(c) ? block_zero_bytes(c.E, c.n_heavy) : 0);
   // Small-block routing kernel: grid-barrier counter (16 B), then a 4-word
   // token bitmask per expert.
   L.cbar = take(16 + (size_t)c.E * 16);
@@ -255,6 +261,29 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
   const int n_part = router_split_parts(c.T, c.d, c.dtype);
   const bool streaming = c.dtype == MOE_BF16 && stream_mlp_supported(c.T);
   bool routed_and_gathered = false;
+  if (moe_block_supported(c)) {
+    // Small bf16 block without a shared expert: the whole layer in one
+    // persistent kernel (router K-sliced over the CTAs, selection, a weight
+    // stream that starts as soon as the experts to stream are known, the
+    // combine). Its sync words, bitmasks, vote totals and counters start
+    // at zero.
+    BlockArgs ba{};
+    MOE_CUDA_TRY(cudaMemsetAsync(at<void>(ws, L.bzero), 0, block_zero_bytes(c.E, c.n_heavy), stream));
+    block_zero_layout(ba, at<void>(ws, L.bzero), c.E);
+    ba.W_r = W_r; ba.part = at<float>(ws, L.rpart);
+    ba.n_slices = block_router_slices(c.d, &ba.kslice);
+    ba.bias = bias; ba.zprev = z_prev; ba.zscale = c.gate_residual_scale;
+    ba.T = c.T; ba.E = c.E; ba.n_heavy = c.n_heavy; ba.k = c.k; ba.routing = c.routing;
+    ba.renorm = c.renorm; ba.M_core = c.M_core;
+    ba.d = c.d; ba.h = c.h; ba.w1_rows_per_group = c.act == MOE_SWIGLU ? 2 * c.h : c.h;
+    ba.x = x; ba.residual = residual; ba.const_vecs = const_vecs; ba.y = y;
+    ba.H = at<void>(ws, L.H); ba.Y = at<void>(ws, L.Y);
+    ba.logits = logits; ba.probs = probs; ba.sel = sel; ba.w = w;
+    ba.votes_out = c.routing == MOE_DES_VOTE ? votes : nullptr; ba.core = core;
+    ba.offsets = offsets; ba.perm = perm; ba.row_of = row_of;
+    ba.dev_status = dev_status;
+    return launch_moe_block(ba, kind_table(c), W1, W2, c.act, stream);
+  }
   if (n_part > 0 && small_route_supported(c.T, c.E, c.k, c.routing, c.dtype)) {
     // Small bf16 block (<= 128 tokens): the router split over the model
     // width, then one cooperative kernel finishes the router, selects (DES:
