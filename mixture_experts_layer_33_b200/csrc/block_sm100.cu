@@ -227,6 +227,17 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
   }
   if (tid < kMaxK) { own_ids[tid] = -1; own_w[tid] = 0.f; }
 
+  // The router's per-expert terms of token t, read now (off the critical path).
+  float zb[kMaxE / 32], zq[kMaxE / 32];
+  if (warp == 0 && t < T) {
+#pragma unroll
+    for (int v = 0; v < kMaxE / 32; ++v) {
+      const int e = lane + 32 * v;
+      zb[v] = (e < E && a.bias) ? __ldg(a.bias + e) : 0.f;
+      zq[v] = (e < E && a.zprev) ? a.zscale * __ldg(a.zprev + (size_t)t * E + e) : 0.f;
+    }
+  }
+
   // ---- 0. router GEMM, K-sliced over the CTAs: CTA s < n_slices computes
   // every token's partial logits over columns [s*kslice, (s+1)*kslice) on
   // the tensor cores (mma.sync m16n8k16, fp32 accumulate), operands staged
@@ -305,22 +316,13 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
 
   // ---- 1. token CTAs finish the router and pick.
   if (t < T && ok_slot) {
-    float zb[kMaxE / 32], zq[kMaxE / 32];
-    if (warp == 0) {
-#pragma unroll
-      for (int v = 0; v < kMaxE / 32; ++v) {
-        const int e = lane + 32 * v;
-        zb[v] = (e < E && a.bias) ? __ldg(a.bias + e) : 0.f;
-        zq[v] = (e < E && a.zprev) ? a.zscale * __ldg(a.zprev + (size_t)t * E + e) : 0.f;
-      }
-    }
     {
       float acc[kMaxE / 32];
 #pragma unroll
       for (int v = 0; v < kMaxE / 32; ++v) acc[v] = 0.f;
       const float *pt = a.part + (size_t)t * E;
       const size_t slice = (size_t)T * E;
-#pragma unroll 4
+#pragma unroll 8
       for (int j = warp; j < a.n_slices; j += kWarps) {
 #pragma unroll
         for (int v = 0; v < kMaxE / 32; ++v) {
@@ -820,12 +822,12 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
       const int s = it / chunks;
       const int c0 = (it - s * chunks) * 256 + lane * 8;
       const bool live = c0 < d;
-      for (int jb = 0; jb < k; jb += 4) {
-        uint4 raw[4];
-        const __nv_bfloat16 *src[4];
-        float wgt[4];
+      for (int jb = 0; jb < k; jb += 8) {  // 8 slots' rows in flight together
+        uint4 raw[8];
+        const __nv_bfloat16 *src[8];
+        float wgt[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 8; ++q) {
           const int j = (jb + q) & 31;
           src[q] = reinterpret_cast<const __nv_bfloat16 *>(
               __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(p.m_src), j));
@@ -836,7 +838,7 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
             raw[q] = l2 ? ld_cg_v4(src[q] + c0) : *reinterpret_cast<const uint4 *>(src[q] + c0);
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 8; ++q)
           if (src[q]) fma8(wgt[q], raw[q], p.acc8);
       }
       if (live) store8(y + (size_t)s * d + c0, p.acc8);
@@ -854,15 +856,24 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
     }
     epi_sync();
     const bool slots_ok = ok_slot != 0;
-    const int it0 = t * 4 + ew;
+    // Items go to warps in the order their CTAs finish their units (a
+    // ticket per warp), so the CTAs that finish first take them.
+    auto claim = [&]() {
+      int it = 0;
+      if (lane == 0) it = (int)atomicAdd(a.sync + 4, 1u);
+      return __shfl_sync(0xffffffffu, it, 0);
+    };
+    const int it0 = slots_ok ? claim() : items;
     Item first;
-    if (slots_ok && it0 < items) prepare(it0, first);
+    if (it0 < items) prepare(it0, first);
     epi_sync();
     if (et == 0)
       ok_slot = (slots_ok && wait_u32(a.sync + 1, (unsigned)G, &abort_flag, a.dev_status)) ? 1 : 0;
     epi_sync();
     if (ok_slot) {
-      for (int it = it0; it < items; it += G * 4) {
+      // With no more items than warps every item went out in the first
+      // round of claims; only claim again when there are more.
+      for (int it = it0; it < items; it = items > 4 * G ? claim() : items) {
         if (it == it0) {
           finish(it, first);
         } else {

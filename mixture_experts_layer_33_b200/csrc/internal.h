@@ -108,7 +108,8 @@ struct BlockArgs {
   int64_t *votes_out;    // DES vote totals for the caller
   int32_t *core, *offsets, *perm, *row_of;
   // The zeroed region (block_zero_bytes), split by block_zero_layout:
-  unsigned *sync;        // [0] barrier arrivals, [1] finished CTAs, [2] unit tickets
+  unsigned *sync;        // [0] barrier arrivals, [1] finished CTAs, [2] unit tickets,
+                         // [3] tokens whose slots are out, [4] combine item tickets
   unsigned *gmask;       // [E][4] token bitmasks
   unsigned long long *votes;  // [E] DES vote totals (exact fixed point)
   int32_t *done;         // [n_heavy] up-unit arrivals per expert

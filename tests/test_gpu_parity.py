@@ -234,6 +234,13 @@ EDGE = [
     ("small_block_des_E128", "des_vote", dict(T=100, d=128, E=128, k=8, h=128, M_core=32)),
     ("small_block_des_T128", "des_vote", dict(T=128, d=256, E=64, k=8, h=128, M_core=16)),
     ("split_router_des_T300", "des_vote", dict(T=300, d=128, E=16, k=4, h=128, M_core=8)),
+    # The whole-layer kernel for small blocks without a shared expert: token
+    # choice with zero-computation experts and the gate residual, the
+    # 128-token boundary, and a model width whose last router slice and
+    # expert widths are ragged (d = 1160, h = 264).
+    ("block_topk_mmoe_kinds", "mmoe", dict(T=96, d=128, h=256, n_shared=0)),
+    ("block_topk_T128", "ditmoe_xl", dict(T=128, d=256, E=16, k=4, h=256, n_shared=0)),
+    ("block_des_ragged_d_h", "des_vote", dict(T=40, d=1160, E=32, k=4, h=264, M_core=12)),
 ]
 
 
