@@ -21,8 +21,10 @@ which is exact). Sources, by page and section:
   Inference, "Conditional Communication": the layer output is the
   routing-score weighted sum of the expert outputs.
 * Dynamic Expert Sharing: Decoupling Memory from Parallelism in
-  Mixture-of-Experts Diffusion LLMs, section 2.4 "DES-Vote" (filter to the
-  own top-K, vote with the routing weights, elect the M_core most voted),
+  Mixture-of-Experts Diffusion LLMs, section 2.3 "DES-Seq" (the core set is
+  the union of every token's top-k_local), section 2.4 "DES-Vote" (filter
+  to the own top-K, vote with the routing weights, elect the M_core most
+  voted),
   section 3.1 (M_core = beta * M) and section 4.3 (tokens re-activate
   experts from the core set at their original per-token count).
 * MMOE: Modernizing Diffusion Transformers with Efficient Expert Design,
@@ -222,6 +224,41 @@ def des_vote(P, K, M_core):
     return votes, core, idx, w
 
 
+def des_seq(P, K, k_local):
+    """DES-Seq core set and restricted re-routing.
+
+    Dynamic Expert Sharing page, section 2.3 "DES-Seq": every token n of the
+    block selects its k_local most salient experts (its top-k_local by P);
+    the core set is the union of these local selections. Section 2.2: the
+    tokens' expert selection is then restricted to the core set; section
+    4.3: at the original per-token count K. Reading: each token takes its
+    min(K, |core|) largest P over the core set, in rank order (ties to the
+    lower id, R6); when the core holds fewer than K experts the remaining
+    slots are empty (expert -1, weight 0). Weights are P itself (R9).
+
+    Returns core [|core|] int32 ascending, idx [N, K] int32, w [N, K].
+    """
+    P = _f64(P)
+    N, M = P.shape
+    if not 1 <= K <= M:
+        raise ValueError("need 1 <= K <= M")
+    if not 1 <= k_local <= M:
+        raise ValueError("need 1 <= k_local <= M")
+    ids = np.arange(M)
+    in_core = np.zeros(M, dtype=bool)
+    for n in range(N):
+        in_core[_order_desc(P[n], ids)[:k_local]] = True
+    core = np.nonzero(in_core)[0].astype(np.int32)
+    idx = np.full((N, K), -1, dtype=np.int32)
+    w = np.zeros((N, K))
+    take = min(K, core.shape[0])
+    for n in range(N):
+        order = _order_desc(P[n, core], core)[:take]
+        idx[n, :take] = core[order]
+        w[n, :take] = P[n, core[order]]
+    return core, idx, w
+
+
 def des_core_size(M, beta):
     """Dynamic Expert Sharing page, section 3.1: M_core = beta * M (floored)."""
     return int(math.floor(float(beta) * M))
@@ -251,7 +288,7 @@ def dispatch(a_tok, a_exp, n_heavy, n_tokens):
     n_assign = a_tok.shape[0]
     counts = np.zeros(n_heavy, dtype=np.int64)
     for a in range(n_assign):
-        if a_exp[a] < n_heavy:
+        if 0 <= a_exp[a] < n_heavy:  # -1: an empty slot (DES-Seq), no row
             counts[a_exp[a]] += 1
     offsets = np.zeros(n_heavy + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(counts)
@@ -260,7 +297,7 @@ def dispatch(a_tok, a_exp, n_heavy, n_tokens):
     row_of = np.full(n_assign, -1, dtype=np.int32)
     for a in range(n_assign):
         e = a_exp[a]
-        if e < n_heavy:
+        if 0 <= e < n_heavy:
             r = fill[e]
             fill[e] += 1
             perm[r] = a_tok[a]
@@ -367,6 +404,8 @@ def combine(tokens, a_tok, a_exp, a_w, expert_out, residual=None,
         if shared_out is not None:
             acc = shared_out[i].copy() if acc is None else acc + shared_out[i]
         for a in np.nonzero(a_tok == s)[0]:
+            if a_exp is not None and a_exp[a] < 0:
+                continue  # an empty slot (DES-Seq) contributes nothing
             term = float(a_w[a]) * expert_out(a)
             acc = term if acc is None else acc + term
         rows.append(acc)
@@ -381,7 +420,7 @@ def assignments_from_selection(cfg, sel):
 
     Token choice / DES: a = s*k + j. Expert choice: a = (g*E + e)*C + c.
     """
-    if cfg["routing"] in ("token_topk", "des_vote"):
+    if cfg["routing"] in ("token_topk", "des_vote", "des_seq"):
         idx = np.asarray(sel["idx"])
         T, k = idx.shape
         a_tok = np.repeat(np.arange(T), k)
@@ -415,6 +454,9 @@ def route(cfg, x, W_r, logit_bias=None, z_prev=None):
     if r == "des_vote":
         votes, core, idx, w = des_vote(A, cfg["k"], cfg["M_core"])
         return {"z": z, "A": A, "votes": votes, "core": core, "idx": idx, "w": w}
+    if r == "des_seq":
+        core, idx, w = des_seq(A, cfg["k"], cfg["k_local"])
+        return {"z": z, "A": A, "core": core, "idx": idx, "w": w}
     raise ValueError(r)
 
 
@@ -448,7 +490,7 @@ def forward(cfg, x, W1, W2, sel, kinds=None, const_vecs=None, Ws1=None,
         if kinds[e] == CONST:
             const_slot[e] = len(const_slot)
     out = {}
-    live = np.nonzero(wanted[a_tok])[0]
+    live = np.nonzero(wanted[a_tok] & (a_exp >= 0))[0]  # -1: empty slot
     for e in np.unique(a_exp[live]):
         rows_a = live[a_exp[live] == e]
         X = _f64(x[a_tok[rows_a]])

@@ -245,6 +245,76 @@ def test_des_core_size_constant_over_block_size():
         assert set(np.unique(idx).tolist()) <= set(core.tolist())
 
 
+def test_des_seq_hand_example():
+    # Two tokens, four experts, local budget 1, K = 2. Token 0 prefers
+    # 2 > 0 > 1 > 3, token 1 prefers 3 > 2 > 0 > 1: core = {2, 3}; token 0
+    # re-routes over the core to (2, 3), token 1 to (3, 2).
+    P = np.array([[0.3, 0.2, 0.4, 0.1], [0.2, 0.1, 0.3, 0.4]])
+    core, idx, w = om.des_seq(P, 2, 1)
+    assert core.tolist() == [2, 3]
+    assert idx.tolist() == [[2, 3], [3, 2]]
+    np.testing.assert_array_equal(w, [[0.4, 0.1], [0.4, 0.3]])
+
+
+def test_des_seq_brute_force_union_and_reroute():
+    rng = np.random.default_rng(21)
+    for N, M, K, kl in [(5, 9, 3, 1), (6, 10, 4, 2), (3, 7, 2, 3), (8, 12, 5, 2)]:
+        P = om.softmax_rows(rng.integers(0, 4, size=(N, M)).astype(float))
+        core, idx, w = om.des_seq(P, K, kl)
+        union = np.zeros(M, dtype=bool)
+        for n in range(N):
+            union |= _rank_mask(P[n], kl)
+        assert np.array_equal(core, np.nonzero(union)[0])
+        take = min(K, len(core))
+        for n in range(N):
+            # brute force: every core expert ranked by (P desc, id asc)
+            ranked = sorted(core.tolist(), key=lambda e: (-P[n, e], e))
+            assert idx[n, :take].tolist() == ranked[:take]
+            assert np.all(idx[n, take:] == -1) and np.all(w[n, take:] == 0)
+            np.testing.assert_array_equal(w[n, :take], P[n, idx[n, :take]])
+
+
+def test_des_seq_local_budget_K_is_vanilla_topk():
+    # k_local = K: every token's own top-K is in the core, so its top-K over
+    # the core is its plain top-K (DES-Seq with the full budget = vanilla).
+    rng = np.random.default_rng(22)
+    P = om.softmax_rows(rng.normal(size=(16, 12)))
+    core, idx, w = om.des_seq(P, 4, 4)
+    assert np.array_equal(idx, om.topk_token_choice(P, 4))
+    assert len(core) <= min(12, 16 * 4)
+
+
+def test_des_seq_local_picks_lead_and_core_bounds():
+    rng = np.random.default_rng(23)
+    M, K = 64, 8
+    for N in (1, 8, 32):
+        for kl in (1, 2, 4):
+            P = om.softmax_rows(rng.normal(size=(N, M)) + rng.normal(size=M)[None])
+            core, idx, _ = om.des_seq(P, K, kl)
+            assert len(core) <= min(M, N * kl)
+            local = om.topk_token_choice(P, kl)
+            assert np.array_equal(idx[:, :kl], local)  # a token's own picks rank first
+            if N == 1:
+                assert core.tolist() == sorted(local[0].tolist())
+                assert np.all(idx[0, kl:] == -1)
+
+
+def test_empty_slots_contribute_nothing():
+    # DES-Seq's empty slots (-1) get no dispatch row and no combine term.
+    cfg = {"routing": "des_seq", "E": 3, "k": 2, "h": 4, "act": "gelu"}
+    rng = np.random.default_rng(24)
+    x = rng.normal(size=(2, 5))
+    W1 = rng.normal(size=(3, 4, 5))
+    W2 = rng.normal(size=(3, 5, 4))
+    full = {"idx": np.array([[1, -1], [0, 2]]), "w": np.array([[0.7, 0.0], [0.4, 0.6]])}
+    y = om.forward(cfg, x, W1, W2, full, residual=x)
+    y0 = x[0] + 0.7 * om.mlp_gelu(x[:1], W1[1], W2[1])[0]
+    np.testing.assert_allclose(y[0], y0, rtol=1e-12)
+    offsets, perm, row_of, _, _ = om.dispatch(np.repeat(np.arange(2), 2),
+                                              full["idx"].reshape(-1), 3, 2)
+    assert offsets.tolist() == [0, 1, 2, 3] and row_of.tolist() == [1, -1, 0, 2]
+
+
 # ---------------------------------------------------------------- dispatch
 def test_dispatch_hand_example():
     # Token choice, T=3, k=2, experts 0..2 heavy, 3 is zero-compute.
