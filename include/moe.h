@@ -4,7 +4,8 @@
  * The layer (shared by DiT-MoE, EC-DiT, MMOE and the DES dLLM block):
  *   router GEMM + softmax      -> affinities A in R^{T x E}
  *   selection                  -> token-choice top-k | expert-choice top-C |
- *                                 DES-Vote core set + restricted top-K
+ *                                 DES-Vote or DES-Seq core set + restricted
+ *                                 top-K
  *   dispatch                   -> stable permutation into per-expert groups
  *   grouped expert MLP         -> GELU or SwiGLU heavy experts (tcgen05 tensor
  *                                 cores for bf16), shared expert(s); the
@@ -69,7 +70,7 @@ enum moe_status {
 #define MOE_DEV_OVERFLOW 8u   /* more rows than the caller's buffers hold */
 
 enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 };
-enum moe_routing { MOE_TOKEN_TOPK = 0, MOE_EXPERT_CHOICE = 1, MOE_DES_VOTE = 2 };
+enum moe_routing { MOE_TOKEN_TOPK = 0, MOE_EXPERT_CHOICE = 1, MOE_DES_VOTE = 2, MOE_DES_SEQ = 3 };
 enum moe_act { MOE_GELU_ERF = 0, MOE_SWIGLU = 1 };
 enum moe_expert_kind { MOE_HEAVY = 0, MOE_IDENTITY = 1, MOE_ZERO = 2, MOE_CONST = 3 };
 
@@ -78,11 +79,11 @@ enum moe_expert_kind { MOE_HEAVY = 0, MOE_IDENTITY = 1, MOE_ZERO = 2, MOE_CONST 
 /*
  * Layer configuration (host memory, read during the call only).
  *
- * T           tokens in the launch (for DES-Vote: the block's N tokens)
+ * T           tokens in the launch (for DES: the block's N tokens)
  * d           model width; h heavy-expert hidden width
  * E           routed experts of every kind (heavy + zero-computation)
  * n_heavy     heavy experts, ids [0, n_heavy)
- * k           token choice: experts per token; DES-Vote: the per-token K
+ * k           token choice: experts per token; DES: the per-token K
  * n_shared, h_shared  shared experts and their hidden width; they are
  *             passed concatenated along the hidden dimension (n_shared *
  *             h_shared hidden units), which for GELU experts equals the sum
@@ -94,6 +95,8 @@ enum moe_expert_kind { MOE_HEAVY = 0, MOE_IDENTITY = 1, MOE_ZERO = 2, MOE_CONST 
  * capacity    expert choice: tokens C chosen per expert per group
  *             (EC-DiT page, "capacity factor": C = f_c * S / E)
  * M_core      DES-Vote core-set size (DES page, section 3.1: beta * M)
+ * k_local     DES-Seq local budget: the core set is the union of every
+ *             token's top-k_local experts (DES page, section 2.3)
  * gate_residual_scale  weight of the previous layer's logits z_prev
  * renorm      0: weights are the full-softmax affinities A (the pages'
  *             definition); 1: renormalised over each token's selection
@@ -107,6 +110,7 @@ typedef struct moe_config {
   int32_t group_size, capacity, M_core;
   float gate_residual_scale;
   int32_t renorm;
+  int32_t k_local;
   int32_t expert_kind[MOE_MAX_EXPERTS];
 } moe_config;
 
@@ -118,7 +122,7 @@ MOE_API const char *moe_status_string(int status);
 MOE_API int moe_device_check(int device);
 
 /* Number of routing assignments of a configuration: T*k for token choice
- * and DES-Vote, (T/S)*E*C for expert choice. */
+ * and DES, (T/S)*E*C for expert choice. */
 MOE_API int moe_num_assignments(const moe_config *cfg, int64_t *n_assign);
 
 /* Workspace bytes moe_forward / moe_forward_host need for `cfg`
@@ -192,6 +196,25 @@ MOE_API int moe_core_set_vote(const float *probs, int N, int M, int K, int M_cor
                       moe_stream_t stream);
 
 /*
+ * DES-Seq core set and restricted re-routing, for one block of N tokens.
+ * Dynamic Expert Sharing page, section 2.3 "DES-Seq": every token selects
+ * its k_local most salient experts (top-k_local by P) and the core set is
+ * the union of these local selections; section 2.2: tokens then select
+ * within the core set, at their original count K (section 4.3).
+ *   probs  [N, M] fp32 in (P = A)
+ *   core   [M] int32 out: the core set in ascending id order, then -1
+ *   n_core [1] int32 out (device): the core-set size
+ *   idx    [N, K] int32 out: each token's min(K, n_core) largest P over the
+ *          core set, descending, ties to the lower id; slots past n_core
+ *          are empty (-1)
+ *   w      [N, K] fp32 out: P[n, idx] (0 for an empty slot)
+ * Limits: 1 <= K <= M <= 256, 1 <= k_local <= M, N <= 4096.
+ */
+MOE_API int moe_core_set_union(const float *probs, int N, int M, int K, int k_local,
+                               int32_t *core, int32_t *n_core, int32_t *idx, float *w,
+                               moe_stream_t stream);
+
+/*
  * Dispatch: a stable permutation of the heavy assignments into per-expert
  * groups (histogram, exclusive scan, scatter), plus the gather of x rows.
  * DICE page, "Conditional Communication" and the expert-parallel
@@ -209,7 +232,9 @@ MOE_API int moe_core_set_vote(const float *probs, int N, int M, int K, int M_cor
  *   x_perm     [n_assign, d] (dtype), nullable: x_perm[r] = x[perm[r]]
  *   tok_ptr    [T + 1], tok_assign [n_assign] int32, nullable, expert choice
  *              only: each token's assignments in slot order (a CSR)
- * Out-of-range ids set MOE_DEV_BAD_EXPERT / MOE_DEV_BAD_TOKEN and are dropped.
+ * Expert id -1 marks an empty slot (DES-Seq with a core smaller than K):
+ * no row, no flag. Other out-of-range ids set MOE_DEV_BAD_EXPERT /
+ * MOE_DEV_BAD_TOKEN and are dropped.
  */
 MOE_API int moe_dispatch(const moe_config *cfg, const int32_t *sel, const void *x,
                  void *x_perm, int32_t *offsets, int32_t *perm, int32_t *row_of,
@@ -311,7 +336,7 @@ typedef struct moe_forward_aux {
   int32_t *sel;      /* [n_assign] idx (token choice, DES) or tok (expert choice) */
   float *w;          /* [n_assign] fp32 routing weights */
   int64_t *votes;    /* [E] DES-Vote only */
-  int32_t *core;     /* [M_core] DES-Vote only */
+  int32_t *core;     /* DES-Vote: [M_core]; DES-Seq: [E], the core set then -1 */
   int32_t *offsets;  /* [n_heavy + 1] */
 } moe_forward_aux;
 

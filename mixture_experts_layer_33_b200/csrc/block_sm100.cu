@@ -175,7 +175,7 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
   __shared__ int core_list[kMaxE];
   __shared__ int glist[kMaxE];  // experts streamed, ascending id
   __shared__ unsigned wbits[kMaxE / 32], sbits[kMaxE / 32];
-  __shared__ int n_groups_s;
+  __shared__ int n_groups_s, n_core_s;
   __shared__ int offs[kMaxE + 1];
   __shared__ unsigned mask[kMaxE][4];  // tokens (<= 128) that picked expert e
   __shared__ int own_ids[kMaxK];
@@ -186,6 +186,8 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
   const int t = blockIdx.x, G = gridDim.x;
   const int T = a.T, E = a.E, k = a.k, nh = a.n_heavy;
   const bool des = a.routing == MOE_DES_VOTE;
+  const bool seq = a.routing == MOE_DES_SEQ;  // DES-Seq: core = union of local top-k_local
+  const bool core_routed = des || seq;         // tokens re-route over a core set
 
   uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~(uintptr_t)1023);
@@ -376,18 +378,22 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
     __syncthreads();
     // Top-k by rank: the candidate (v, e) takes slot #{f : v_f > v or
     // (v_f == v and f < e)} if below k (the picks and order of repeated
-    // argmax with ties to the lower id). DES ranks P and votes with it;
+    // argmax with ties to the lower id). DES-Vote ranks P and votes with
+    // its top-K; DES-Seq ranks P and marks its top-k_local in the union;
     // token choice ranks the logits, weight P.
     if (tid < E) {
       const int e = tid;
-      const float *key = des ? As : zs;
+      const float *key = core_routed ? As : zs;
       const float ke = key[e];
       int rank = 0;
       for (int f = 0; f < E; ++f) {
         const float kf = key[f];
         rank += (kf > ke) || (kf == ke && f < e);
       }
-      if (rank < k) {
+      if (seq) {
+        if (rank < a.k_local)
+          atomicOr(reinterpret_cast<unsigned *>(a.votes) + (e >> 5), 1u << (e & 31));
+      } else if (rank < k) {
         if (des) {
           atomicAdd(a.votes + e, (unsigned long long)vote_quantum(As[e]));
         } else {
@@ -397,7 +403,7 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
         }
       }
     }
-    if (!des && a.renorm) {
+    if (!core_routed && a.renorm) {
       __syncthreads();
       if (tid == 0) {
         float ws = 0.f;
@@ -432,6 +438,8 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
         }
         in = rank < a.M_core;
       }
+    } else if (seq) {
+      if (tid < E) in = (__ldcg(reinterpret_cast<const unsigned *>(a.votes) + (tid >> 5)) >> (tid & 31)) & 1u;
     } else {
       for (int i = tid; i < 4 * nh; i += kThreads) (&mask[0][0])[i] = __ldcg(a.gmask + i);
       __syncthreads();
@@ -446,12 +454,22 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
       if (lane == 0) { wbits[warp] = b; sbits[warp] = bs; }
     }
     __syncthreads();
-    if (in && des) {
+    if (in && core_routed) {
       int pos = __popc(wbits[warp] & ((1u << lane) - 1u));
       for (int w = 0; w < warp; ++w) pos += __popc(wbits[w]);
       core_list[pos] = tid;
       if (t == 0) a.core[pos] = tid;
     }
+    if (tid == 0) {
+      int n = 0;
+#pragma unroll
+      for (int w = 0; w < kMaxE / 32; ++w) n += __popc(wbits[w]);
+      n_core_s = n;
+    }
+    __syncthreads();
+    // DES-Seq's core list is as long as the union: the rest of the caller's
+    // core array reads -1.
+    if (seq && t == 0 && tid >= n_core_s && tid < E) a.core[tid] = -1;
     if (streamed) {
       int pos = __popc(sbits[warp] & ((1u << lane) - 1u));
       for (int w = 0; w < warp; ++w) pos += __popc(sbits[w]);
@@ -613,10 +631,12 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
     const int et = tid - 64;  // 0..127
     const int ew = et >> 5;   // 0..3
     bool ok = true;
-    if (des) {
+    if (core_routed) {
       // Re-route the own token over the core set, by rank (the core list
-      // ascends, so a lower position is a lower id), and mark the picks.
-      const int Mc = a.M_core;
+      // ascends, so a lower position is a lower id), and mark the picks:
+      // min(K, |core|) of them (DES-Seq's core can be smaller than K; the
+      // other slots stay empty).
+      const int Mc = des ? a.M_core : n_core_s;
       if (t < T && et < Mc) {
         const int e = core_list[et];
         const float p = As[e];
@@ -664,7 +684,9 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
         const int j = et, i = t * k + j;
         const int e = own_ids[j];
         int row = -1;
-        if (e < 0 || e >= E) {
+        if (e == -1) {
+          // an empty slot (DES-Seq with a core smaller than K)
+        } else if (e < 0 || e >= E) {
           set_status(a.dev_status, MOE_DEV_BAD_EXPERT);
         } else if (e < nh) {
           const int q = t >> 5;
@@ -929,7 +951,8 @@ int run_block(const BlockArgs &a, const KindTable &kinds, const void *W1, const 
 }  // namespace
 
 bool moe_block_supported(const moe_config &c) {
-  return c.dtype == MOE_BF16 && (c.routing == MOE_TOKEN_TOPK || c.routing == MOE_DES_VOTE) &&
+  return c.dtype == MOE_BF16 &&
+         (c.routing == MOE_TOKEN_TOPK || c.routing == MOE_DES_VOTE || c.routing == MOE_DES_SEQ) &&
          c.T >= 1 && c.T <= 128 && c.T < num_sms() && c.E >= 1 && c.E <= kMaxE && c.k >= 1 &&
          c.k <= kMaxK && c.n_shared == 0 && c.n_heavy >= 0 && c.h >= 8 && c.d >= 8 &&
          c.d <= 32768;

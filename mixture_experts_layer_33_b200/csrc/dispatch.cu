@@ -34,6 +34,7 @@ __device__ __forceinline__ bool decode(const DispatchArgs &a, int64_t i, int &to
   } else {
     tok = (int)(i / a.k);
     exp = a.sel[i];
+    if (exp == -1) return false;  // an empty slot (DES-Seq): no row, no flag
     if (exp < 0 || exp >= a.E) {
       set_status(a.dev_status, MOE_DEV_BAD_EXPERT);
       return false;

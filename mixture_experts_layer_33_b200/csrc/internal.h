@@ -94,7 +94,7 @@ struct BlockArgs {
   int n_slices, kslice;  // router K slices over the CTAs, columns per slice
   const float *bias, *zprev;
   float zscale;
-  int T, E, n_heavy, k, routing, renorm, M_core;
+  int T, E, n_heavy, k, routing, renorm, M_core, k_local;
   int d, h;              // model width, expert hidden width
   int w1_rows_per_group; // h (GELU) or 2h (SwiGLU: gate rows, then up rows)
   const void *x;         // [T][d] bf16
@@ -111,7 +111,7 @@ struct BlockArgs {
   unsigned *sync;        // [0] barrier arrivals, [1] finished CTAs, [2] unit tickets,
                          // [3] tokens whose slots are out, [4] combine item tickets
   unsigned *gmask;       // [E][4] token bitmasks
-  unsigned long long *votes;  // [E] DES vote totals (exact fixed point)
+  unsigned long long *votes;  // [E] DES-Vote totals (exact fixed point); DES-Seq: core bitmask
   int32_t *done;         // [n_heavy] up-unit arrivals per expert
   int32_t *dev_status;
 };
@@ -134,6 +134,9 @@ int launch_expert_choice(const float *probs, int T, int E, int S, int C,
 int launch_des_reroute(const float *probs, const int64_t *votes, int N, int M, int K,
                        int M_core, int32_t *core, int32_t *idx, float *w,
                        cudaStream_t stream);
+// DES-Seq: core = union of every token's top-k_local; restricted re-route.
+int launch_des_seq(const float *probs, int N, int M, int K, int k_local, int32_t *core,
+                   int32_t *n_core, int32_t *idx, float *w, cudaStream_t stream);
 int launch_des_vote(const float *probs, int N, int M, int K, int M_core,
                     int64_t *votes, int32_t *core, int32_t *idx, float *w,
                     cudaStream_t stream);

@@ -54,6 +54,10 @@ int check_config(const moe_config *c) {
       if (c->k < 1 || c->k > c->M_core || c->M_core > c->E) return MOE_ERR_INVALID_ARG;
       if (c->T > 4096) return MOE_ERR_UNSUPPORTED;
       break;
+    case MOE_DES_SEQ:
+      if (c->k < 1 || c->k > c->E || c->k_local < 1 || c->k_local > c->E) return MOE_ERR_INVALID_ARG;
+      if (c->T > 4096) return MOE_ERR_UNSUPPORTED;
+      break;
     default:
       return MOE_ERR_INVALID_ARG;
   }
@@ -274,7 +278,7 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
     ba.n_slices = block_router_slices(c.d, &ba.kslice);
     ba.bias = bias; ba.zprev = z_prev; ba.zscale = c.gate_residual_scale;
     ba.T = c.T; ba.E = c.E; ba.n_heavy = c.n_heavy; ba.k = c.k; ba.routing = c.routing;
-    ba.renorm = c.renorm; ba.M_core = c.M_core;
+    ba.renorm = c.renorm; ba.M_core = c.M_core; ba.k_local = c.k_local;
     ba.d = c.d; ba.h = c.h; ba.w1_rows_per_group = c.act == MOE_SWIGLU ? 2 * c.h : c.h;
     ba.x = x; ba.residual = residual; ba.const_vecs = const_vecs; ba.y = y;
     ba.H = at<void>(ws, L.H); ba.Y = at<void>(ws, L.Y);
@@ -313,7 +317,7 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
     st = launch_small_route(sa, stream);
     if (st != MOE_OK) return st;
     routed_and_gathered = true;
-  } else if (n_part > 0 && c.routing != MOE_EXPERT_CHOICE) {
+  } else if (n_part > 0 && (c.routing == MOE_TOKEN_TOPK || c.routing == MOE_DES_VOTE)) {
     // Small bf16 block: router split over the model width, then a per-token
     // finish that also selects (token choice) or sums the exact int64 DES
     // votes (cleared by the split router); DES then elects the core set and
@@ -334,6 +338,9 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
       st = launch_expert_choice(probs, c.T, c.E, c.group_size, c.capacity, sel, w, stream);
     else if (c.routing == MOE_DES_VOTE)
       st = launch_des_vote(probs, c.T, c.E, c.k, c.M_core, votes, core, sel, w, stream);
+    else if (c.routing == MOE_DES_SEQ)  // the core-set size goes to the (unused) vote slot
+      st = launch_des_seq(probs, c.T, c.E, c.k, c.k_local, core,
+                          reinterpret_cast<int32_t *>(at<int64_t>(ws, L.votes)), sel, w, stream);
     if (st != MOE_OK) return st;
   }
   if (!routed_and_gathered) {
@@ -458,6 +465,14 @@ int moe_core_set_vote(const float *probs, int N, int M, int K, int M_core, int64
   if (M > MOE_MAX_EXPERTS || N > 4096) return MOE_ERR_UNSUPPORTED;
   if (!probs || !votes || !core || !idx || !w) return MOE_ERR_INVALID_ARG;
   return launch_des_vote(probs, N, M, K, M_core, votes, core, idx, w, stream);
+}
+
+int moe_core_set_union(const float *probs, int N, int M, int K, int k_local, int32_t *core,
+                       int32_t *n_core, int32_t *idx, float *w, moe_stream_t stream) {
+  if (N < 0 || M < 1 || K < 1 || K > M || k_local < 1 || k_local > M) return MOE_ERR_INVALID_ARG;
+  if (M > MOE_MAX_EXPERTS || N > 4096) return MOE_ERR_UNSUPPORTED;
+  if (!probs || !core || !n_core || !idx || !w) return MOE_ERR_INVALID_ARG;
+  return launch_des_seq(probs, N, M, K, k_local, core, n_core, idx, w, stream);
 }
 
 int moe_dispatch(const moe_config *cfg, const int32_t *sel, const void *x, void *x_perm,

@@ -280,7 +280,113 @@ des_reroute_kernel(const float *__restrict__ P, const int64_t *__restrict__ vote
   }
 }
 
+// DES-Seq for one block of N tokens, one CTA: every token's top-k_local by
+// P marks the core set (a bitmask); the core list ascends; each token then
+// takes its min(K, |core|) largest P over the core, the rest empty (-1).
+template <int kDesVpl>
+__global__ void __launch_bounds__(kDesThreads)
+des_seq_kernel(const float *__restrict__ P, int N, int M, int K, int kl,
+               int32_t *__restrict__ core, int32_t *__restrict__ n_core,
+               int32_t *__restrict__ idx, float *__restrict__ w) {
+  __shared__ unsigned bits[MOE_MAX_EXPERTS / 32];
+  __shared__ int in_core[MOE_MAX_EXPERTS];
+  __shared__ int ncore_s;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
+  if (tid < MOE_MAX_EXPERTS / 32) bits[tid] = 0u;
+  __syncthreads();
+  for (int n = warp; n < N; n += nwarps) {
+    float p[kDesVpl];
+    bool taken[kDesVpl];
+#pragma unroll
+    for (int v = 0; v < kDesVpl; ++v) {
+      const int e = lane + 32 * v;
+      p[v] = e < M ? P[(size_t)n * M + e] : -INFINITY;
+      taken[v] = false;
+    }
+    for (int r = 0; r < kl; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int v = 0; v < kDesVpl; ++v) {
+        const int e = lane + 32 * v;
+        if (e < M && !taken[v] && better(p[v], e, bv, bi)) { bv = p[v]; bi = e; }
+      }
+      warp_argmax(bv, bi);
+#pragma unroll
+      for (int v = 0; v < kDesVpl; ++v)
+        if (lane + 32 * v == bi) {
+          taken[v] = true;
+          atomicOr(&bits[bi >> 5], 1u << (bi & 31));
+        }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < M; e += blockDim.x) {
+    const bool in = (bits[e >> 5] >> (e & 31)) & 1u;
+    in_core[e] = in;
+    if (in) {
+      int pos = __popc(bits[e >> 5] & ((1u << (e & 31)) - 1u));
+      for (int q = 0; q < (e >> 5); ++q) pos += __popc(bits[q]);
+      core[pos] = e;
+    }
+  }
+  if (tid == 0) {
+    int c = 0;
+    for (int q = 0; q < (M + 31) / 32; ++q) c += __popc(bits[q]);
+    ncore_s = c;
+    *n_core = c;
+  }
+  __syncthreads();
+  const int nc = ncore_s;
+  for (int e = nc + tid; e < M; e += blockDim.x) core[e] = -1;
+  const int take = nc < K ? nc : K;
+  for (int n = warp; n < N; n += nwarps) {
+    float p[kDesVpl];
+    bool taken[kDesVpl];
+#pragma unroll
+    for (int v = 0; v < kDesVpl; ++v) {
+      const int e = lane + 32 * v;
+      const bool ok = e < M && in_core[e];
+      p[v] = ok ? P[(size_t)n * M + e] : -INFINITY;
+      taken[v] = !ok;
+    }
+    for (int r = 0; r < K; ++r) {
+      int bi = -1;
+      float pw = 0.f;
+      if (r < take) {
+        float bv = -INFINITY;
+        bi = 0x7fffffff;
+#pragma unroll
+        for (int v = 0; v < kDesVpl; ++v) {
+          const int e = lane + 32 * v;
+          if (!taken[v] && better(p[v], e, bv, bi)) { bv = p[v]; bi = e; }
+        }
+        warp_argmax(bv, bi);
+        float own = 0.f;
+#pragma unroll
+        for (int v = 0; v < kDesVpl; ++v)
+          if (lane + 32 * v == bi) { taken[v] = true; own = p[v]; }
+        pw = __shfl_sync(0xffffffffu, own, bi & 31);
+      }
+      if (lane == 0) {
+        idx[(size_t)n * K + r] = bi;
+        w[(size_t)n * K + r] = pw;
+      }
+    }
+  }
+}
+
 }  // namespace
+
+int launch_des_seq(const float *probs, int N, int M, int K, int k_local, int32_t *core,
+                   int32_t *n_core, int32_t *idx, float *w, cudaStream_t stream) {
+  if (M <= 32) des_seq_kernel<1><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, k_local, core, n_core, idx, w);
+  else if (M <= 64) des_seq_kernel<2><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, k_local, core, n_core, idx, w);
+  else if (M <= 128) des_seq_kernel<4><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, k_local, core, n_core, idx, w);
+  else des_seq_kernel<8><<<1, kDesThreads, 0, stream>>>(probs, N, M, K, k_local, core, n_core, idx, w);
+  return last_launch_status();
+}
 
 int launch_expert_choice(const float *probs, int T, int E, int S, int C, int32_t *tok,
                          float *w, cudaStream_t stream) {

@@ -67,6 +67,13 @@ MMOE_SKEW_BIAS = 0.791
 WORKLOADS["mmoe_skewed"] = dict(WORKLOADS["mmoe"], zero_compute_logit_bias=MMOE_SKEW_BIAS)
 
 
+# The DES page's two core-set functions and the vanilla block on the same
+# inputs (seed 3): DES-Seq (section 2.3) with a local budget of 2 experts
+# per token, and vanilla top-8 routing with no core set (section 2.5).
+WORKLOADS["des_seq"] = dict(WORKLOADS["des_vote"], routing="des_seq", k_local=2)
+WORKLOADS["des_vanilla"] = dict(WORKLOADS["des_vote"], routing="token_topk")
+
+
 def workload(name, **overrides):
     """The named workload's configuration, with shape overrides applied."""
     cfg = copy.deepcopy(WORKLOADS[name])

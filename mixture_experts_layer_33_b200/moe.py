@@ -18,7 +18,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so"
 
 MOE_OK = 0
 F32, BF16 = 0, 1
-TOKEN_TOPK, EXPERT_CHOICE, DES_VOTE = 0, 1, 2
+TOKEN_TOPK, EXPERT_CHOICE, DES_VOTE, DES_SEQ = 0, 1, 2, 3
 GELU_ERF, SWIGLU = 0, 1
 HEAVY, IDENTITY, ZERO, CONST = 0, 1, 2, 3
 DEV_BAD_EXPERT, DEV_BAD_TOKEN, DEV_TIMEOUT, DEV_OVERFLOW = 1, 2, 4, 8
@@ -28,7 +28,7 @@ MAX_EXPERTS = 256
 ENTRY_POINTS = (
     "moe_status_string", "moe_device_check", "moe_num_assignments",
     "moe_workspace_size", "moe_router", "moe_select_topk",
-    "moe_select_expert_choice", "moe_core_set_vote", "moe_dispatch",
+    "moe_select_expert_choice", "moe_core_set_vote", "moe_core_set_union", "moe_dispatch",
     "moe_grouped_mlp", "moe_combine", "moe_forward", "moe_forward_host",
     "moe_dispatch_noalloc", "moe_activation",
 )
@@ -43,6 +43,7 @@ class MoeConfig(ctypes.Structure):
         ("dtype", ctypes.c_int32), ("act", ctypes.c_int32), ("routing", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("capacity", ctypes.c_int32), ("M_core", ctypes.c_int32),
         ("gate_residual_scale", ctypes.c_float), ("renorm", ctypes.c_int32),
+        ("k_local", ctypes.c_int32),
         ("expert_kind", ctypes.c_int32 * MAX_EXPERTS),
     ]
 
@@ -64,6 +65,7 @@ _SIGS = {
     "moe_select_topk": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_select_expert_choice": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_core_set_vote": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "moe_core_set_union": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_dispatch": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_dispatch_noalloc": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_activation": (_i32, [_vp, _vp, ctypes.c_int64, _i32, _vp]),
@@ -136,12 +138,13 @@ def make_config(cfg) -> MoeConfig:
     c.dtype = BF16 if cfg["dtype"] == "bf16" else F32
     c.act = SWIGLU if cfg["act"] == "swiglu" else GELU_ERF
     c.routing = {"token_topk": TOKEN_TOPK, "expert_choice": EXPERT_CHOICE,
-                 "des_vote": DES_VOTE}[cfg["routing"]]
+                 "des_vote": DES_VOTE, "des_seq": DES_SEQ}[cfg["routing"]]
     c.group_size = cfg.get("group_size", 0)
     c.capacity = cfg.get("capacity", 0)
     c.M_core = cfg.get("M_core", 0)
     c.gate_residual_scale = float(cfg.get("gate_residual_scale", 0.0))
     c.renorm = int(cfg.get("renorm", 0))
+    c.k_local = int(cfg.get("k_local", 0))
     for e, k in enumerate(kinds):
         c.expert_kind[e] = k
     return c
@@ -198,6 +201,13 @@ def core_set_vote(probs, K, M_core, votes, core, idx, w, stream=None):
     _check(LIB.moe_core_set_vote(_dev_ptr(probs), N, M, int(K), int(M_core), _dev_ptr(votes),
                                  _dev_ptr(core), _dev_ptr(idx), _dev_ptr(w), _stream(stream)),
            "moe_core_set_vote")
+
+
+def core_set_union(probs, K, k_local, core, n_core, idx, w, stream=None):
+    N, M = probs.shape
+    _check(LIB.moe_core_set_union(_dev_ptr(probs), N, M, int(K), int(k_local), _dev_ptr(core),
+                                  _dev_ptr(n_core), _dev_ptr(idx), _dev_ptr(w), _stream(stream)),
+           "moe_core_set_union")
 
 
 def dispatch(c: MoeConfig, sel, x, x_perm, offsets, perm, row_of, tok_ptr, tok_assign,

@@ -42,7 +42,8 @@ def run_layer(cfg, inp, device="cuda"):
         "sel": torch.empty(na, dtype=torch.int32, device=dev),
         "w": torch.empty(na, dtype=torch.float32, device=dev),
         "votes": torch.empty(E, dtype=torch.int64, device=dev),
-        "core": torch.empty(max(cfg.get("M_core", 0), 1), dtype=torch.int32, device=dev),
+        "core": torch.empty(E if cfg["routing"] == "des_seq" else max(cfg.get("M_core", 0), 1),
+                            dtype=torch.int32, device=dev),
         "offsets": torch.empty(c.n_heavy + 1, dtype=torch.int32, device=dev),
     }
     ws = m.alloc_workspace(c, dev)
@@ -83,6 +84,9 @@ def oracle_selection_from_gpu(cfg, out):
     if r == "expert_choice":
         tok, w = oracle.expert_choice(A, cfg["group_size"], cfg["capacity"])
         return {"tok": tok, "w": w}
+    if r == "des_seq":
+        core, idx, w = oracle.des_seq(A, cfg["k"], cfg["k_local"])
+        return {"idx": idx, "w": w, "core": core}
     votes, core, idx, w = oracle.des_vote(A, cfg["k"], cfg["M_core"])
     return {"idx": idx, "w": w, "votes": votes, "core": core}
 

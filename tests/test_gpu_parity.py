@@ -60,6 +60,10 @@ def _check_selection(cfg, out):
     if cfg["routing"] == "des_vote":
         np.testing.assert_array_equal(out["votes"], ref["votes"])
         np.testing.assert_array_equal(out["core"][:cfg["M_core"]], ref["core"])
+    if cfg["routing"] == "des_seq":
+        nc = len(ref["core"])
+        np.testing.assert_array_equal(out["core"][:nc], ref["core"])
+        assert np.all(out["core"][nc:] == -1)
     a_tok, a_exp, _ = oracle.assignments_from_selection(cfg, gpu)
     offsets, *_ = oracle.dispatch(a_tok, a_exp, cfg["E_heavy"], cfg["T"])
     np.testing.assert_array_equal(out["offsets"], offsets)
@@ -241,6 +245,13 @@ EDGE = [
     ("block_topk_mmoe_kinds", "mmoe", dict(T=96, d=128, h=256, n_shared=0)),
     ("block_topk_T128", "ditmoe_xl", dict(T=128, d=256, E=16, k=4, h=256, n_shared=0)),
     ("block_des_ragged_d_h", "des_vote", dict(T=40, d=1160, E=32, k=4, h=264, M_core=12)),
+    # DES-Seq (core = union of local top-k_local): the whole-layer kernel,
+    # a core smaller than K (one token: empty slots), the full local
+    # budget (= vanilla), and the general path past 128 tokens.
+    ("block_des_seq", "des_seq", dict(d=256, h=256)),
+    ("block_des_seq_one_token", "des_seq", dict(T=1, d=256, h=256)),
+    ("block_des_seq_full_budget", "des_seq", dict(T=16, d=256, h=256, k_local=8)),
+    ("des_seq_T300_general_path", "des_seq", dict(T=300, d=128, E=16, k=4, h=128, k_local=1)),
 ]
 
 
@@ -261,6 +272,30 @@ def test_edge_cases(label, name, over):
         assert int(out["offsets"][-1]) == 0  # no heavy rows: no GEMM tiles at all
 
 
+@pytest.mark.parametrize("N,kl", [(32, 2), (1, 2), (64, 1), (300, 3)])
+def test_core_set_union_entry_point(N, kl):
+    """moe_core_set_union against the oracle's DES-Seq on the GPU's own probabilities."""
+    m = H.moe()
+    cfg = gen.workload("des_seq", T=N, d=128, h=128, k_local=kl)
+    inp = gen.make_inputs(cfg, "cuda")
+    T, E, K = cfg["T"], cfg["E"], cfg["k"]
+    logits = torch.empty(T, E, device="cuda")
+    probs = torch.empty(T, E, device="cuda")
+    m.router(inp["x"], inp["W_r"], logits, probs, bias=inp["logit_bias"])
+    core = torch.empty(E, dtype=torch.int32, device="cuda")
+    n_core = torch.empty(1, dtype=torch.int32, device="cuda")
+    idx = torch.empty(T, K, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, K, device="cuda")
+    m.core_set_union(probs, K, kl, core, n_core, idx, w)
+    torch.cuda.synchronize()
+    ref_core, ref_idx, ref_w = oracle.des_seq(probs.cpu().numpy().astype(np.float64), K, kl)
+    assert int(n_core.item()) == len(ref_core)
+    np.testing.assert_array_equal(core.cpu().numpy()[:len(ref_core)], ref_core)
+    assert np.all(core.cpu().numpy()[len(ref_core):] == -1)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
+    np.testing.assert_array_equal(w.cpu().numpy().astype(np.float64), ref_w)
+
+
 def test_deterministic_bytes():
     cfg = gen.workload("mmoe", T=600, d=256, h=512, h_shared=256)
     inp = gen.make_inputs(cfg, "cuda")
@@ -279,7 +314,7 @@ def test_bad_indices_are_flagged_not_faulted():
     g = torch.Generator(device="cpu").manual_seed(5)
     sel = torch.randint(0, cfg["E"], (na,), generator=g, dtype=torch.int32)
     sel[3] = 99
-    sel[10] = -1
+    sel[10] = -2  # (-1 marks an empty slot and is skipped without a flag)
     sel = sel.cuda()
     x = torch.randn(cfg["T"], cfg["d"], device="cuda").to(torch.bfloat16)
     ws = m.alloc_workspace(c)
