@@ -65,9 +65,9 @@ NCU_TRAFFIC = {
 def fused_block(cfg):
     """Whether moe_forward runs this layer as one persistent kernel (the
     library's rule for small blocks: bf16, at most 128 tokens, token choice
-    or DES-Vote, no shared expert, E <= 128, k <= 32, d <= 32768)."""
+    or DES, no shared expert, E <= 128, k <= 32, d <= 32768)."""
     return (cfg["dtype"] == "bf16" and 1 <= cfg["T"] <= 128
-            and cfg["routing"] in ("token_topk", "des_vote") and cfg["n_shared"] == 0
+            and cfg["routing"] in ("token_topk", "des_vote", "des_seq") and cfg["n_shared"] == 0
             and cfg["E"] <= 128 and cfg["k"] <= 32 and cfg["d"] <= 32768)
 
 
@@ -85,7 +85,7 @@ def forward_launches(cfg):
     if (bf16 and cfg["T"] <= 128 and r in ("token_topk", "des_vote") and cfg["E"] <= 128
             and cfg["k"] <= 32 and cfg["T"] * cfg["k"] <= 2048):
         return n + 2  # split router, then routing + dispatch + gather in one kernel
-    if bf16 and cfg["T"] <= 512 and not ec:
+    if bf16 and cfg["T"] <= 512 and r in ("token_topk", "des_vote"):
         n += 2 + (r == "des_vote")  # split router, finish (+ DES re-route)
     else:
         n += 1 + (r != "token_topk")  # router (+ expert choice / DES vote)
@@ -109,6 +109,8 @@ def describe(cfg):
         parts.append(f"top-{cfg['k']}")
     elif cfg["routing"] == "expert_choice":
         parts.append(f"expert-choice S={cfg['group_size']} C={cfg['capacity']}")
+    elif cfg["routing"] == "des_seq":
+        parts.append(f"DES-Seq K={cfg['k']} k_local={cfg['k_local']}")
     else:
         parts.append(f"DES-Vote K={cfg['k']} M_core={cfg['M_core']}")
     parts.append(f"h={cfg['h']} {cfg['act']}")
@@ -269,6 +271,8 @@ class StagedLayer:
         self.w = torch.empty(na, dtype=torch.float32, **f)
         self.votes = torch.empty(E, dtype=torch.int64, **f)
         self.core = torch.empty(max(1, cfg.get("M_core", 0)), dtype=torch.int32, **f)
+        self.core_all = torch.empty(E, dtype=torch.int32, **f)  # DES-Seq: the union, then -1
+        self.n_core = torch.empty(1, dtype=torch.int32, **f)
         self.offsets = torch.empty(self.c.n_heavy + 1, dtype=torch.int32, **f)
         self.perm = torch.empty(na, dtype=torch.int32, **f)
         self.row_of = torch.empty(na, dtype=torch.int32, **f)
@@ -325,6 +329,9 @@ class StagedLayer:
             m.select_expert_choice(self.probs, cfg["group_size"], cfg["capacity"], self.sel, self.w)
         elif r == "des_vote":
             m.core_set_vote(self.probs, cfg["k"], cfg["M_core"], self.votes, self.core, self.sel, self.w)
+        elif r == "des_seq":
+            m.core_set_union(self.probs, cfg["k"], cfg["k_local"], self.core_all, self.n_core,
+                             self.sel, self.w)
         mark(1)
         m.dispatch(self.c, self.sel, i["x"], self.x_perm, self.offsets, self.perm, self.row_of,
                    self.tok_ptr, self.tok_assign, self.status, self.ws)
@@ -477,7 +484,7 @@ def gpu_bench(args):
     tr = NCU_TRAFFIC.get(cfg["name"])
     traffic = tr["bytes"] if tr and tr["sha256_16"] == source_hash(tr["source"]) else None
     gm_ms = stage_ms["grouped_mlp"] / args.steps  # grouped-MLP launches, from timed region 2
-    if cfg["routing"] == "des_vote":
+    if cfg["dtype"] == "bf16" and cfg["T"] <= 128:  # small blocks stream expert weights
         bytes_ = weight_bytes_used(cfg, used)
         if fused_ms is not None:
             kname = "moe_block_kernel (whole layer, one launch after a memset)"
@@ -620,6 +627,75 @@ def reference_bench(args):
     print(json.dumps(line), flush=True)
 
 
+def des_sweep(args):
+    """DES page, sections 3.3 and 4.2: the small block under vanilla top-8,
+    DES-Seq and DES-Vote, for blocks of N = 8..64 tokens on the skewed
+    synthetic logits. Per N and routing: U (experts that get rows, so
+    weights read), the layer time (moe_forward as a CUDA graph, L2
+    flushed clean before every step) and U * 12.58 MB / time. One JSON line;
+    not part of the driver's contract."""
+    import torch
+
+    from mixture_experts_layer_33_b200 import inputs as gen
+    from mixture_experts_layer_33_b200 import moe as m
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = L2Flush(dev)
+    variants = [("vanilla top-8", "des_vanilla", {}),
+                ("DES-Seq k_local=1", "des_seq", {"k_local": 1}),
+                ("DES-Seq k_local=2", "des_seq", {"k_local": 2}),
+                ("DES-Vote beta=0.5", "des_vote", {})]
+    rows = []
+    for N in (8, 16, 32, 64):
+        for label, name, over in variants:
+            cfg = gen.workload(name, T=N, **over)
+            inp = gen.make_inputs(cfg, dev)
+            c = m.make_config(cfg)
+            ws = m.alloc_workspace(c, dev)
+            y = torch.empty_like(inp["x"])
+            status = torch.zeros(1, dtype=torch.int32, device=dev)
+            offsets = torch.empty(c.n_heavy + 1, dtype=torch.int32, device=dev)
+
+            def fwd(aux=None):
+                m.forward(c, inp["x"], inp["W_r"], inp["W1"], inp["W2"], y, ws,
+                          residual=inp["x"], bias=inp["logit_bias"], aux=aux,
+                          dev_status=status)
+            fwd({"offsets": offsets})
+            torch.cuda.synchronize()
+            offs = offsets.cpu().tolist()
+            U = sum(1 for a, b in zip(offs[:-1], offs[1:]) if b > a)
+            for _ in range(args.warmup):
+                fwd()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fwd()
+            times = []
+            for s in range(args.steps):
+                flush(s)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                b.synchronize()
+                times.append(a.elapsed_time(b) * 1e3)
+            del g
+            if int(status.item()) != 0:
+                raise RuntimeError(f"device status {int(status.item())} for {label} N={N}")
+            us = statistics.median(times)
+            wbytes = U * 3 * cfg["d"] * cfg["h"] * 2
+            rows.append({"N": N, "routing": label, "U": U, "layer_us": round(us, 1),
+                         "weight_gbs": round(wbytes / (us / 1e6) / 1e9, 1)})
+    for N in (8, 16, 32, 64):
+        van = next(r for r in rows if r["N"] == N and r["routing"].startswith("vanilla"))
+        for r in rows:
+            if r["N"] == N:
+                r["latency_vs_vanilla"] = round(r["layer_us"] / van["layer_us"], 3)
+    print(json.dumps({"sweep": "DES block: vanilla vs DES-Seq vs DES-Vote",
+                      "workload": describe(gen.workload("des_vote")), "steps": args.steps,
+                      "l2": "flushed clean before every step", "rows": rows}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -630,10 +706,14 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
+    ap.add_argument("--des-sweep", action="store_true",
+                    help="vanilla vs DES-Seq vs DES-Vote over block sizes (one JSON line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.des_sweep:
+        des_sweep(args)
+    elif args.impl == "reference":
         reference_bench(args)
     else:
         gpu_bench(args)

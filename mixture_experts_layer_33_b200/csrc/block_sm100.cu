@@ -174,7 +174,7 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
   __shared__ long long V[kMaxE];
   __shared__ int core_list[kMaxE];
   __shared__ int glist[kMaxE];  // experts streamed, ascending id
-  __shared__ unsigned wbits[kMaxE / 32], sbits[kMaxE / 32];
+  __shared__ unsigned wbits[kMaxE / 32], sbits[kMaxE / 32], lbits[kMaxE / 32];
   __shared__ int n_groups_s, n_core_s;
   __shared__ int offs[kMaxE + 1];
   __shared__ unsigned mask[kMaxE][4];  // tokens (<= 128) that picked expert e
@@ -447,11 +447,17 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
     }
     // The core set (DES) and the experts to stream (its heavy members; for
     // token choice the heavy experts some token picked), ascending id.
+    // Streamed first: experts certain to get rows; last: DES-Vote core
+    // members without votes, which get rows only in corner cases (their
+    // units are skipped if the routing shows no rows by the time they are
+    // claimed).
     const bool streamed = in && tid < nh;
+    const bool late = streamed && des && V[tid] == 0;
     if (tid < kMaxE) {
       const unsigned b = __ballot_sync(0xffffffffu, in);
-      const unsigned bs = __ballot_sync(0xffffffffu, streamed);
-      if (lane == 0) { wbits[warp] = b; sbits[warp] = bs; }
+      const unsigned bs = __ballot_sync(0xffffffffu, streamed && !late);
+      const unsigned bl = __ballot_sync(0xffffffffu, late);
+      if (lane == 0) { wbits[warp] = b; sbits[warp] = bs; lbits[warp] = bl; }
     }
     __syncthreads();
     if (in && core_routed) {
@@ -471,15 +477,18 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
     // core array reads -1.
     if (seq && t == 0 && tid >= n_core_s && tid < E) a.core[tid] = -1;
     if (streamed) {
-      int pos = __popc(sbits[warp] & ((1u << lane) - 1u));
-      for (int w = 0; w < warp; ++w) pos += __popc(sbits[w]);
+      const unsigned *bits = late ? lbits : sbits;
+      int pos = __popc(bits[warp] & ((1u << lane) - 1u));
+      for (int w = 0; w < warp; ++w) pos += __popc(bits[w]);
+      if (late)
+        for (int w = 0; w < kMaxE / 32; ++w) pos += __popc(sbits[w]);
       glist[pos] = tid;
     }
     if (des && t == 0 && tid < E && a.votes_out) a.votes_out[tid] = V[tid];
     if (tid == 0) {
       int n = 0;
 #pragma unroll
-      for (int w = 0; w < kMaxE / 32; ++w) n += __popc(sbits[w]);
+      for (int w = 0; w < kMaxE / 32; ++w) n += __popc(sbits[w]) + __popc(lbits[w]);
       n_groups_s = n;
     }
   }
@@ -513,11 +522,20 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
         // hand its id to the MMA and epilogue warps; -1 ends the list.
         int u = (int)atomicAdd(a.sync + 2, 1u);
         if (u >= total) u = -1;
+        int code = u;
+        if (u >= 0 && route_ready) {
+          __threadfence_block();  // the offsets written before the flag
+          // The routing is known: an expert that got no rows needs no
+          // weights (the unit is passed on as skipped: -2 - u).
+          const int g0 = u < n_up ? glist[u / up_blocks] : glist[(u - n_up) / down_blocks];
+          if (offs[g0 + 1] == offs[g0]) code = -2 - u;
+        }
         if (!mbar_wait(uqe0 + 8 * qs, qph ^ 1u, &abort_flag, a.dev_status)) { ok = false; break; }
-        uq[qs] = u;
+        uq[qs] = code;
         mbar_arrive(uqf0 + 8 * qs);
         if (++qs == kUQ) { qs = 0; qph ^= 1u; }
         if (u < 0) break;
+        if (code < -1) continue;
         const bool up = u < n_up;
         const int g = up ? glist[u / up_blocks] : glist[(u - n_up) / down_blocks];
         const int blk = up ? u % up_blocks : (u - n_up) % down_blocks;
@@ -530,6 +548,7 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
           // complete once all of the expert's up units are stored.
           if (!routed) {
             if (!wait_local(&route_ready, &abort_flag, a.dev_status)) { ok = false; break; }
+            __threadfence_block();  // the offsets written before the flag
             routed = true;
           }
           if (!wait_s32(a.done + g, 4 * up_blocks, &abort_flag, a.dev_status)) { ok = false; break; }
@@ -582,7 +601,8 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
         if (!mbar_wait(uqf0 + 8 * qs, qph, &abort_flag, a.dev_status)) break;
         const int u = uq[qs];
         if (++qs == kUQ) { qs = 0; qph ^= 1u; }
-        if (u < 0) break;
+        if (u == -1) break;
+        if (u < -1) continue;  // skipped unit: no MMA
         const bool up = u < n_up;
         const int K = up ? a.d : a.h;
         const int nkb = (K + BK - 1) / BK;
@@ -719,10 +739,22 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
     while (ok) {
       const bool got = mbar_wait(uqf0 + 8 * qs, qph, &abort_flag, a.dev_status);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      const int u = uq[qs];
+      const int code = uq[qs];
       const uint32_t uq_done = uqe0 + 8 * qs;
       if (++qs == kUQ) { qs = 0; qph ^= 1u; }
-      if (u < 0) break;
+      if (code == -1) break;
+      if (code < -1) {
+        // Skipped unit (its expert got no rows): nothing to store, but an
+        // up unit still counts toward its expert's arrivals.
+        const int su = -2 - code;
+        __syncwarp();
+        if (lane == 0) {
+          if (su < n_up) atomicAdd(a.done + glist[su / up_blocks], 1);
+          mbar_arrive(uq_done);
+        }
+        continue;
+      }
+      const int u = code;
       const bool up = u < n_up;
       const int g = up ? glist[u / up_blocks] : glist[(u - n_up) / down_blocks];
       const int blk = up ? u % up_blocks : (u - n_up) % down_blocks;
