@@ -696,6 +696,71 @@ def des_sweep(args):
                       "l2": "flushed clean before every step", "rows": rows}), flush=True)
 
 
+def ec_sweep(args):
+    """EC-DiT page, "Expert-Choice routing" and "capacity factor": the
+    expert-choice layer (T=8192, d=2048, E=32, h=8192) with the routing
+    group per sequence (S=128) or the whole batch (S=8192) and capacity
+    factors f_c in {1, 2, 4} (C = f_c*S/E). Per variant: layer time, grouped
+    MLP TFLOP/s and the histogram of experts per token (a token may get 0
+    or several experts under expert choice). One JSON line; not part of the
+    driver's contract."""
+    import torch
+
+    from mixture_experts_layer_33_b200 import inputs as gen
+    from mixture_experts_layer_33_b200 import moe as m
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = L2Flush(dev)
+    rows = []
+    for S in (128, 8192):
+        for fc in (1, 2, 4):
+            C = fc * S // 32
+            cfg = gen.workload("ecdit", group_size=S, capacity=C)
+            inp = gen.make_inputs(cfg, dev)
+            c = m.make_config(cfg)
+            na = m.num_assignments(c)
+            ws = m.alloc_workspace(c, dev)
+            y = torch.empty_like(inp["x"])
+            status = torch.zeros(1, dtype=torch.int32, device=dev)
+            sel = torch.empty(na, dtype=torch.int32, device=dev)
+
+            def fwd(aux=None):
+                m.forward(c, inp["x"], inp["W_r"], inp["W1"], inp["W2"], y, ws,
+                          residual=inp["x"], aux=aux, dev_status=status)
+            fwd({"sel": sel})
+            torch.cuda.synchronize()
+            per_token = torch.bincount(sel.long(), minlength=cfg["T"]).cpu()
+            hist = torch.bincount(per_token).tolist()
+            for _ in range(args.warmup):
+                fwd()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fwd()
+            times = []
+            for s_ in range(args.steps):
+                flush(s_)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                g.replay()
+                b.record()
+                b.synchronize()
+                times.append(a.elapsed_time(b))
+            del g, ws
+            if int(status.item()) != 0:
+                raise RuntimeError(f"device status {int(status.item())} for S={S} f_c={fc}")
+            ms = statistics.median(times)
+            flops = mlp_flops(cfg, na)
+            rows.append({"S": S, "f_c": fc, "C": C, "assignments": na, "layer_ms": round(ms, 4),
+                         "tokens_per_s": round(cfg["T"] / (ms / 1e3), 1),
+                         "layer_tflops": round(flops / (ms / 1e3) / 1e12, 1),
+                         "experts_per_token_hist": hist})
+            torch.cuda.empty_cache()
+    print(json.dumps({"sweep": "EC-DiT expert choice: routing group x capacity factor",
+                      "workload": describe(gen.workload("ecdit")), "steps": args.steps,
+                      "l2": "flushed clean before every step", "rows": rows}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -708,11 +773,15 @@ def main(argv=None):
     ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
     ap.add_argument("--des-sweep", action="store_true",
                     help="vanilla vs DES-Seq vs DES-Vote over block sizes (one JSON line)")
+    ap.add_argument("--ec-sweep", action="store_true",
+                    help="expert choice: routing group x capacity factor (one JSON line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
     if args.des_sweep:
         des_sweep(args)
+    elif args.ec_sweep:
+        ec_sweep(args)
     elif args.impl == "reference":
         reference_bench(args)
     else:

@@ -65,6 +65,10 @@ WORKLOADS = {
 # tests/golden/calibrate_mmoe_skew.py.
 MMOE_SKEW_BIAS = 0.791
 WORKLOADS["mmoe_skewed"] = dict(WORKLOADS["mmoe"], zero_compute_logit_bias=MMOE_SKEW_BIAS)
+# Late blocks: 23.4 % of the routing to the lightweight experts (same page,
+# same calibration).
+MMOE_LATE_BIAS = 0.2351
+WORKLOADS["mmoe_late"] = dict(WORKLOADS["mmoe"], zero_compute_logit_bias=MMOE_LATE_BIAS)
 
 
 # The DES page's two core-set functions and the vanilla block on the same

@@ -33,7 +33,8 @@ PAIR = [
     ("ecdit", dict(T=32 * 128, group_size=128, d=256, E=8, h=512, capacity=32)),
     ("des_vote", dict(T=1024, d=256, E=16, k=4, h=256, M_core=8)),
 ]
-FULL = ["tiny_fp32", "ditmoe_xl", "ecdit", "des_vote", "mmoe", "mmoe_skewed"]
+FULL = ["tiny_fp32", "ditmoe_xl", "ecdit", "des_vote", "mmoe", "mmoe_skewed", "mmoe_late",
+        "des_seq", "des_vanilla"]
 
 
 def _check_router(cfg, hin, out):
@@ -227,6 +228,9 @@ EDGE = [
     ("all_zero_compute", "mmoe", dict(T=200, d=128, h=256, h_shared=128, zero_compute_logit_bias=60.0)),
     ("ec_full_capacity", "ecdit", dict(T=64, group_size=16, d=128, E=4, h=256, capacity=16)),
     ("ec_whole_batch", "ecdit", dict(T=2048, group_size=2048, d=128, E=8, h=256, capacity=512)),
+    # capacity factors f_c = 1 and 4 (C = f_c * S / E with S = 128, E = 8)
+    ("ec_capacity_factor_1", "ecdit", dict(T=512, group_size=128, d=128, E=8, h=256, capacity=16)),
+    ("ec_capacity_factor_4", "ecdit", dict(T=512, group_size=128, d=128, E=8, h=256, capacity=64)),
     ("des_beta_one", "des_vote", dict(d=128, h=128, M_core=64)),
     ("odd_N_swiglu_routed", "des_vote", dict(T=37, d=128, E=16, k=4, h=128, M_core=8)),
     ("tiny_fp32_k1", "tiny_fp32", dict(k=1)),

@@ -504,3 +504,19 @@ def test_planted_vote_without_filter_is_caught():
     P = np.array(g["P"])
     unfiltered = (P * 2.0 ** 40).sum(axis=0)
     assert int(np.argmax(unfiltered)) == 0 and unfiltered[3] != g["votes_real"][3] * 2 ** 40
+
+
+@pytest.mark.parametrize("name,share", [("mmoe_skewed", 0.446), ("mmoe_late", 0.234)])
+def test_mmoe_lightweight_shares(name, share):
+    # MMOE page, "routing analysis": 44.6 % (early blocks) and 23.4 % (late
+    # blocks) of the routing goes to the lightweight experts. The workloads'
+    # biases reproduce those shares under the oracle's own routing.
+    from mixture_experts_layer_33_b200 import inputs as gen
+    cfg = gen.workload(name, T=2048)
+    inp = gen.make_inputs(cfg, "cpu")
+    hin = {k: gen.to_numpy_f32(inp[k]) if inp[k] is not None else None
+           for k in ("x", "W_r", "logit_bias", "z_prev")}
+    z = om.router_logits(hin["x"], hin["W_r"], hin["logit_bias"], hin["z_prev"],
+                         cfg["gate_residual_scale"])
+    idx = om.topk_token_choice(z, cfg["k"])
+    assert abs(float(np.mean(idx >= cfg["E_heavy"])) - share) < 0.02
