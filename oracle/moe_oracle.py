@@ -355,11 +355,14 @@ def mlp_swiglu(X, Wg, Wu, Wd):
     return H @ _f64(Wd).T
 
 
-def zero_compute_expert(kind, X, v=None):
+def zero_compute_expert(kind, X, v=None, Wc=None):
     """MMOE zero-computation experts: identity -> x, zero -> 0, constant -> v.
 
     The constant expert returns its learned vector v [d] for every token
-    (reading R14).
+    (reading R14). Mixture variant (MMOE page, "Methodology": a constant
+    expert mixes with a learned vector; reading R24): with learned mixing
+    weights Wc [2, d], E(x) = a0(x) * x + a1(x) * v where
+    (a0, a1) = softmax(Wc . x).
     """
     X = _f64(X)
     if kind == IDENTITY:
@@ -367,7 +370,11 @@ def zero_compute_expert(kind, X, v=None):
     if kind == ZERO:
         return np.zeros_like(X)
     if kind == CONST:
-        return np.broadcast_to(_f64(v)[None, :], X.shape).copy()
+        v = _f64(v)
+        if Wc is None:
+            return np.broadcast_to(v[None, :], X.shape).copy()
+        a = softmax_rows(X @ _f64(Wc).T)  # [rows, 2]
+        return a[:, :1] * X + a[:, 1:2] * v[None, :]
     raise ValueError("not a zero-computation kind")
 
 
@@ -467,8 +474,10 @@ def forward(cfg, x, W1, W2, sel, kinds=None, const_vecs=None, Ws1=None,
     ``W1`` [E_h, h, d] (GELU) or [E_h, 2h, d] (SwiGLU, gate then up rows),
     ``W2`` [E_h, d, h]. ``kinds`` [E] gives each expert's kind (heavy ids
     come first); ``const_vecs`` [n_const, d] holds the constant experts'
-    vectors in id order. Shared experts arrive concatenated along the hidden
-    dimension: ``Ws1`` [n_sh*h_sh, d], ``Ws2`` [d, n_sh*h_sh]; for GELU
+    vectors in id order, or [n_const, 3, d] (v, then the two rows of the
+    mixing weights Wc) when ``cfg["const_mix"]`` is set. Shared experts
+    arrive concatenated along the hidden dimension: ``Ws1`` [n_sh*h_sh, d],
+    ``Ws2`` [d, n_sh*h_sh]; for GELU
     this is the sum of the individual shared experts exactly (the hidden
     units of different experts never mix).
 
@@ -497,7 +506,11 @@ def forward(cfg, x, W1, W2, sel, kinds=None, const_vecs=None, Ws1=None,
         if kinds[e] == HEAVY:
             Y = heavy_expert(cfg["act"], X, W1[e], W2[e], h)
         elif kinds[e] == CONST:
-            Y = zero_compute_expert(CONST, X, const_vecs[const_slot[e]])
+            cv = const_vecs[const_slot[e]]
+            if cfg.get("const_mix"):
+                Y = zero_compute_expert(CONST, X, cv[0], cv[1:3])
+            else:
+                Y = zero_compute_expert(CONST, X, cv)
         else:
             Y = zero_compute_expert(int(kinds[e]), X)
         for i, a in enumerate(rows_a):
@@ -527,7 +540,9 @@ def dense_masked_forward(cfg, x, W1, W2, A, mask, kinds=None,
         if kinds[e] == HEAVY:
             Ye = heavy_expert(cfg["act"], x64, W1[e], W2[e], cfg["h"])
         elif kinds[e] == CONST:
-            Ye = zero_compute_expert(CONST, x64, const_vecs[ci])
+            cv = const_vecs[ci]
+            Ye = (zero_compute_expert(CONST, x64, cv[0], cv[1:3]) if cfg.get("const_mix")
+                  else zero_compute_expert(CONST, x64, cv))
             ci += 1
         else:
             Ye = zero_compute_expert(int(kinds[e]), x64)

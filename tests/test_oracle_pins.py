@@ -520,3 +520,41 @@ def test_mmoe_lightweight_shares(name, share):
                          cfg["gate_residual_scale"])
     idx = om.topk_token_choice(z, cfg["k"])
     assert abs(float(np.mean(idx >= cfg["E_heavy"])) - share) < 0.02
+
+
+def test_constant_mixture_closed_forms():
+    # Mixture variant of the constant expert: E(x) = a0 x + a1 v with
+    # (a0, a1) = softmax(Wc x). Zero mixing weights give the midpoint; a
+    # dominant first (second) logit gives x (v); a hand-computed case.
+    rng = np.random.default_rng(31)
+    X = rng.normal(size=(3, 4))
+    v = rng.normal(size=4)
+    mid = om.zero_compute_expert(om.CONST, X, v, np.zeros((2, 4)))
+    np.testing.assert_allclose(mid, 0.5 * X + 0.5 * v[None], rtol=1e-15)
+    big = np.zeros((2, 4))
+    big[0, 0] = 800.0
+    Xp = np.abs(X) + 1.0  # x_0 > 0: logit0 = 800 x_0 dominates
+    np.testing.assert_allclose(om.zero_compute_expert(om.CONST, Xp, v, big), Xp, rtol=1e-12)
+    np.testing.assert_allclose(om.zero_compute_expert(om.CONST, Xp, v, -big),
+                               np.broadcast_to(v, Xp.shape), rtol=1e-12)
+    x1 = np.array([[1.0, 2.0]])
+    Wc = np.array([[0.5, 0.0], [0.0, 0.5]])     # logits (0.5, 1.0)
+    a0 = 1.0 / (1.0 + math.exp(0.5))            # softmax of (0.5, 1.0), first entry
+    got = om.zero_compute_expert(om.CONST, x1, np.array([3.0, -1.0]), Wc)
+    np.testing.assert_allclose(got, [[a0 * 1 + (1 - a0) * 3, a0 * 2 + (1 - a0) * -1]], rtol=1e-14)
+    # without mixing weights: the plain learned vector (reading R14)
+    np.testing.assert_array_equal(om.zero_compute_expert(om.CONST, X, v), np.broadcast_to(v, X.shape))
+
+
+def test_constant_mixture_routes_through_layer():
+    # Every token routed (top-1, weight 1 after renorm) to the mixed constant
+    # expert: y = x + E_c(x).
+    cfg = {"routing": "token_topk", "E": 2, "k": 1, "h": 4, "act": "gelu", "const_mix": 1}
+    rng = np.random.default_rng(32)
+    x = rng.normal(size=(5, 6))
+    cv = rng.normal(size=(1, 3, 6))
+    sel = {"idx": np.ones((5, 1), dtype=np.int32), "w": np.ones((5, 1))}
+    y = om.forward(cfg, x, np.zeros((1, 4, 6)), np.zeros((1, 6, 4)), sel,
+                   kinds=[om.HEAVY, om.CONST], const_vecs=cv, residual=x)
+    a = om.softmax_rows(x @ cv[0, 1:3].T)
+    np.testing.assert_allclose(y, x + a[:, :1] * x + a[:, 1:2] * cv[0, 0][None], rtol=1e-13)
