@@ -97,6 +97,10 @@ enum moe_expert_kind { MOE_HEAVY = 0, MOE_IDENTITY = 1, MOE_ZERO = 2, MOE_CONST 
  * M_core      DES-Vote core-set size (DES page, section 3.1: beta * M)
  * k_local     DES-Seq local budget: the core set is the union of every
  *             token's top-k_local experts (DES page, section 2.3)
+ * const_mix   0: a constant expert returns its learned vector v; 1: it
+ *             returns a0 x + a1 v with (a0, a1) = softmax(Wc x) (MMOE
+ *             page, "Methodology": a learned-vector mixture); const_vecs
+ *             then holds [n_const, 3, d]: v, then the two rows of Wc
  * gate_residual_scale  weight of the previous layer's logits z_prev
  * renorm      0: weights are the full-softmax affinities A (the pages'
  *             definition); 1: renormalised over each token's selection
@@ -111,6 +115,7 @@ typedef struct moe_config {
   float gate_residual_scale;
   int32_t renorm;
   int32_t k_local;
+  int32_t const_mix;
   int32_t expert_kind[MOE_MAX_EXPERTS];
 } moe_config;
 
@@ -302,11 +307,14 @@ MOE_API int moe_grouped_mlp(const moe_config *cfg, const void *x_perm,
  *         w[a] * { y_perm[row_of[a]] (heavy), x_s (identity), 0 (zero),
  *                  const_vecs[c] (c-th constant expert) }
  * summed in fp32 and rounded once to dtype. y_perm, y_shared are in dtype.
+ * With cfg->const_mix a constant expert's term is a0 x_s + a1 v_c,
+ * (a0, a1) = softmax(Wc_c x_s); its x part is added after the slots.
  * `residual` may be the same buffer as `y` (the sum is formed element by
  * element before y is written).
  *   sel, w       the selection (as in moe_dispatch) and its [n_assign] weights
  *   row_of       from moe_dispatch;  tok_ptr/tok_assign: expert choice only
- *   x            [T, d] (identity experts); const_vecs [n_const, d], nullable
+ *   x            [T, d] (identity experts); const_vecs [n_const, d]
+ *                ([n_const, 3, d] with const_mix), nullable
  *   residual     [T, d] nullable (r = 0);  y [T, d] out (dtype)
  */
 MOE_API int moe_combine(const moe_config *cfg, const void *y_perm,

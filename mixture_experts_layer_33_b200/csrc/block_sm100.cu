@@ -987,6 +987,7 @@ bool moe_block_supported(const moe_config &c) {
          (c.routing == MOE_TOKEN_TOPK || c.routing == MOE_DES_VOTE || c.routing == MOE_DES_SEQ) &&
          c.T >= 1 && c.T <= 128 && c.T < num_sms() && c.E >= 1 && c.E <= kMaxE && c.k >= 1 &&
          c.k <= kMaxK && c.n_shared == 0 && c.n_heavy >= 0 && c.h >= 8 && c.d >= 8 &&
+         c.const_mix == 0 &&
          c.d <= 32768;
 }
 

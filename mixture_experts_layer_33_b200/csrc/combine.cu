@@ -56,6 +56,31 @@ template <> struct Raw8<float> {
   }
 };
 
+// (a0, a1) = softmax(Wc . x) of a mixed constant expert, Wc = rows 1..2 of
+// its [3, d] block `vrow`; fp32 dot products by the whole warp. Out of
+// line: the rare path keeps its registers to itself.
+template <typename T>
+__device__ __noinline__ float2 const_mix_weights(const T *xr, const T *vrow, int d) {
+  const int lane = threadIdx.x & 31;
+  float z0 = 0.f, z1 = 0.f;
+  for (int c = lane * 8; c < d; c += 256) {
+    float xv[8], w0[8], w1[8];
+    load8(xr + c, xv);
+    load8(vrow + d + c, w0);
+    load8(vrow + 2 * d + c, w1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      z0 = fmaf(xv[i], w0[i], z0);
+      z1 = fmaf(xv[i], w1[i], z1);
+    }
+  }
+  z0 = warp_sum(z0);
+  z1 = warp_sum(z1);
+  const float mz = fmaxf(z0, z1);
+  const float e0 = expf(z0 - mz), e1 = expf(z1 - mz);
+  return make_float2(e0 / (e0 + e1), e1 / (e0 + e1));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTable kinds) {
   const T *__restrict__ x = static_cast<const T *>(a.x);
@@ -88,6 +113,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += t[i];
     }
+    float x_coef = 0.f;  // weight of x_s from mixed constant experts
     for (int j0 = a0; j0 < a1; j0 += 32) {
       // Lane j holds slot j0 + j: its weight and the first element of its
       // source row (the expert's output row, x for an identity expert, the
@@ -95,6 +121,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
       // the dispatch dropped, or an id it flagged).
       const T *m_src = nullptr;
       float m_w = 0.f;
+      bool m_mix = false;
       if (j0 + lane < a1) {
         const int asg = ec ? a.tok_assign[j0 + lane] : j0 + lane;
         const int e = ec ? (int)((asg / a.C) % a.E) : a.sel[asg];
@@ -107,10 +134,24 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
           } else if (kind == MOE_IDENTITY) {
             m_src = x + (size_t)s * a.d;
           } else if (kind == MOE_CONST) {
-            m_src = cv + (size_t)kinds.cidx[e] * a.d;
+            m_src = cv + (size_t)kinds.cidx[e] * (a.const_mix ? 3 : 1) * a.d;
+            m_mix = a.const_mix != 0;
           }
           m_w = wv;
         }
+      }
+      // Mixed constant experts: the warp forms (a0, a1) = softmax(Wc x_s)
+      // for each such slot; the slot keeps w * a1 on v, and w * a0 joins
+      // the coefficient of x_s, added after the slots.
+      for (unsigned mm = __ballot_sync(0xffffffffu, m_mix); mm; mm &= mm - 1u) {
+        const int j = __ffs(mm) - 1;
+        const T *vrow = reinterpret_cast<const T *>(
+            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(m_src), j));
+        const float2 mix = const_mix_weights(x + (size_t)s * a.d, vrow, a.d);
+        const float a0 = mix.x, a1 = mix.y;
+        const float wj = __shfl_sync(0xffffffffu, m_w, j);
+        x_coef = fmaf(wj, a0, x_coef);
+        if (lane == j) m_w = wj * a1;
       }
       const int nj = min(32, a1 - j0);
       for (int jb = 0; jb < nj; jb += kBatch) {
@@ -130,6 +171,11 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
         for (int u = 0; u < kBatch; ++u)
           if (src[u]) raw[u].fma_into(wgt[u], acc);
       }
+    }
+    if (live && x_coef != 0.f) {
+      Raw8<T> xs;
+      xs.load(x + (size_t)s * a.d + c0);
+      xs.fma_into(x_coef, acc);
     }
     if (live) store8(y + (size_t)s * a.d + c0, acc);
   }

@@ -62,6 +62,7 @@ int check_config(const moe_config *c) {
       return MOE_ERR_INVALID_ARG;
   }
   if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_INVALID_ARG;
+  if (c->const_mix != 0 && c->const_mix != 1) return MOE_ERR_INVALID_ARG;
   if (n_assign_of(*c) > (int64_t)0x7fffffff) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -234,7 +235,7 @@ CombineArgs combine_args(const moe_config &c, const void *y_perm, const void *y_
                          int32_t *dev_status) {
   CombineArgs a;
   a.routing = c.routing; a.T = c.T; a.d = c.d; a.E = c.E; a.k = c.k;
-  a.S = c.group_size; a.C = c.capacity; a.dtype = c.dtype;
+  a.S = c.group_size; a.C = c.capacity; a.dtype = c.dtype; a.const_mix = c.const_mix;
   a.y_perm = y_perm; a.y_shared = y_shared; a.sel = sel; a.w = w; a.row_of = row_of;
   a.tok_ptr = tok_ptr; a.tok_assign = tok_assign; a.x = x; a.const_vecs = const_vecs;
   a.residual = residual; a.y = y; a.dev_status = dev_status;

@@ -22,7 +22,7 @@ HEAVY, IDENTITY, ZERO, CONST = 0, 1, 2, 3
 
 # Tensor ids of the per-tensor generator streams.
 _TID = {"x": 1, "W_r": 2, "W1": 3, "W2": 4, "Ws1": 5, "Ws2": 6,
-        "logit_bias": 7, "z_prev": 8, "const_vecs": 9}
+        "logit_bias": 7, "z_prev": 8, "const_vecs": 9, "const_mix": 10}
 
 # The five workloads. Shapes and distributions follow the pages' models:
 #   tiny_fp32  - small token-choice layer (fp32) for exhaustive checks;
@@ -69,6 +69,9 @@ WORKLOADS["mmoe_skewed"] = dict(WORKLOADS["mmoe"], zero_compute_logit_bias=MMOE_
 # same calibration).
 MMOE_LATE_BIAS = 0.2351
 WORKLOADS["mmoe_late"] = dict(WORKLOADS["mmoe"], zero_compute_logit_bias=MMOE_LATE_BIAS)
+# The constant expert as a learned-vector mixture (a0 x + a1 v, (a0, a1) =
+# softmax(Wc x)), on the early-block routing so that it gets many tokens.
+WORKLOADS["mmoe_constmix"] = dict(WORKLOADS["mmoe_skewed"], const_mix=1)
 
 
 # The DES page's two core-set functions and the vanilla block on the same
@@ -127,7 +130,8 @@ def make_inputs(cfg, device="cpu"):
       W2         [E_h, d, h]
       Ws1        [n_sh*h_sh, d] or None (shared experts, concatenated hidden)
       Ws2        [d, n_sh*h_sh] or None
-      const_vecs [n_const, d] or None   (constant experts' vectors, id order)
+      const_vecs [n_const, d] or None   (constant experts' vectors, id order;
+                 [n_const, 3, d] with const_mix: v, then the mixing weights Wc)
     """
     dt = torch_dtype(cfg)
     T, d, E, h = cfg["T"], cfg["d"], cfg["E"], cfg["h"]
@@ -159,6 +163,10 @@ def make_inputs(cfg, device="cpu"):
     n_const = sum(1 for k in cfg["kinds"] if k == CONST)
     out["const_vecs"] = (_normal((n_const, d), ws, "const_vecs", cfg, device, dt)
                          if n_const else None)
+    if n_const and cfg.get("const_mix"):
+        # [n_const, 3, d]: v, then the mixing weights Wc [2, d]
+        wc = _normal((n_const, 2, d), ws, "const_mix", cfg, device, dt)
+        out["const_vecs"] = torch.cat([out["const_vecs"][:, None, :], wc], dim=1).contiguous()
     return out
 
 

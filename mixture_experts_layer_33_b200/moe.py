@@ -43,7 +43,7 @@ class MoeConfig(ctypes.Structure):
         ("dtype", ctypes.c_int32), ("act", ctypes.c_int32), ("routing", ctypes.c_int32),
         ("group_size", ctypes.c_int32), ("capacity", ctypes.c_int32), ("M_core", ctypes.c_int32),
         ("gate_residual_scale", ctypes.c_float), ("renorm", ctypes.c_int32),
-        ("k_local", ctypes.c_int32),
+        ("k_local", ctypes.c_int32), ("const_mix", ctypes.c_int32),
         ("expert_kind", ctypes.c_int32 * MAX_EXPERTS),
     ]
 
@@ -145,6 +145,7 @@ def make_config(cfg) -> MoeConfig:
     c.gate_residual_scale = float(cfg.get("gate_residual_scale", 0.0))
     c.renorm = int(cfg.get("renorm", 0))
     c.k_local = int(cfg.get("k_local", 0))
+    c.const_mix = int(cfg.get("const_mix", 0))
     for e, k in enumerate(kinds):
         c.expert_kind[e] = k
     return c

@@ -26,6 +26,7 @@ SMALL = [
     ("des_vote", dict(d=256, h=256)),
     ("mmoe", dict(T=600, d=256, h=512, h_shared=256)),
     ("mmoe_skewed", dict(T=600, d=256, h=512, h_shared=256)),
+    ("mmoe_constmix", dict(T=600, d=256, h=512, h_shared=256)),
 ]
 # Groups averaging >= 256 rows: the grouped GEMM runs on two-SM (M=256) tiles.
 PAIR = [
@@ -34,7 +35,7 @@ PAIR = [
     ("des_vote", dict(T=1024, d=256, E=16, k=4, h=256, M_core=8)),
 ]
 FULL = ["tiny_fp32", "ditmoe_xl", "ecdit", "des_vote", "mmoe", "mmoe_skewed", "mmoe_late",
-        "des_seq", "des_vanilla"]
+        "mmoe_constmix", "des_seq", "des_vanilla"]
 
 
 def _check_router(cfg, hin, out):
@@ -247,6 +248,9 @@ EDGE = [
     # 128-token boundary, and a model width whose last router slice and
     # expert widths are ragged (d = 1160, h = 264).
     ("block_topk_mmoe_kinds", "mmoe", dict(T=96, d=128, h=256, n_shared=0)),
+    # mixed constant experts on a small block (the general path) and fp32
+    ("small_constmix_no_shared", "mmoe_constmix", dict(T=96, d=128, h=256, n_shared=0)),
+    ("constmix_fp32", "mmoe_constmix", dict(T=200, d=64, h=128, h_shared=64, dtype="f32")),
     ("block_topk_T128", "ditmoe_xl", dict(T=128, d=256, E=16, k=4, h=256, n_shared=0)),
     ("block_des_ragged_d_h", "des_vote", dict(T=40, d=1160, E=32, k=4, h=264, M_core=12)),
     # DES-Seq (core = union of local top-k_local): the whole-layer kernel,
