@@ -367,9 +367,22 @@ MOE_API int moe_forward(const moe_config *cfg, const void *x, const void *residu
 /*
  * moe_forward with the activations in HOST memory: copies x_host (and
  * residual_host, z_prev_host if given) to the device, runs the layer and
- * copies y back to y_host, all enqueued on `stream`. Weights stay device
- * pointers. For the copies to be asynchronous the host buffers should be
- * pinned; the caller synchronises `stream` before reading y_host.
+ * copies y back to y_host. Weights stay device pointers. For the copies to
+ * be asynchronous the host buffers should be pinned; the caller
+ * synchronises `stream` before reading y_host.
+ *
+ * Batches of at least 4096 tokens (token or expert choice) run as a
+ * pipeline of 2 or 3 token chunks: chunk i's layer runs on `stream` while
+ * chunk i+1 is copied in on one library-owned side stream and chunk i-1 is
+ * copied out on another. The side streams fork from `stream` at entry and
+ * join it before return, so work enqueued on `stream` afterwards sees y_host
+ * complete, as in the one-chunk form. Chunks are whole routing units (whole
+ * groups for expert choice; a DES block is never cut) and every later step
+ * is per row or per token, so y is bit-identical to the unchunked layer.
+ * Calls on a stream under CUDA graph capture take the one-chunk form. The
+ * side streams and their events are made on first use per device and live
+ * until process exit; concurrent callers serialise on a host mutex while
+ * they enqueue.
  */
 MOE_API int moe_forward_host(const moe_config *cfg, const void *x_host,
                      const void *residual_host, const float *z_prev_host,

@@ -2,6 +2,8 @@
 // orchestration of the layer's kernels (declared in include/moe.h).
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -142,6 +144,108 @@ T *at(void *ws, size_t off) {
 int check_ws(const moe_config &c, void *ws, size_t ws_bytes) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < layout_of(c).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// ---- host path: chunked copy / compute pipeline
+
+constexpr int kHostMaxChunks = 4;
+constexpr int64_t kHostMinChunkTokens = 2048;
+// Relative chunk sizes: a small first chunk starts the layer early and a
+// small last chunk ends the copy-out early. A chunk costs a fixed part (the
+// fixed-latency kernels, the GEMMs' last wave, one more pass over the
+// expert weights) on top of its per-token share, which bounds how many pay
+// off: the third one re-reads the weights at HBM speed (~6.5 TB/s) to hide
+// about a quarter of the activations' copies at PCIe speed (~55 GB/s each
+// way), so it is taken while the weights stay under ~30x the activations.
+constexpr int kHostPlan2[] = {1, 1};
+constexpr int kHostPlan3[] = {1, 2, 1};
+constexpr double kHostThirdChunkRatio = 30.0;
+
+// Expert weight bytes one pass of the layer reads (routed and shared).
+double layer_weight_bytes(const moe_config &c) {
+  const double w1_rows = c.act == MOE_SWIGLU ? 2.0 * c.h : c.h;
+  const double hs = (double)c.n_shared * c.h_shared;  // Ws1 [hs, d], Ws2 [d, hs]
+  return ((double)c.n_heavy * (w1_rows + c.h) + 2.0 * hs) * c.d * elem_bytes(c.dtype);
+}
+
+// Chunk boundaries of moe_forward_host's token pipeline: bounds[0] = 0 <
+// bounds[1] < ... < bounds[n] = T; returns n (1: no pipelining). A chunk is
+// a whole number of routing units: token choice routes each token on its
+// own (any cut; 128-token multiples keep the GEMM tiles full), expert
+// choice routes whole groups, and DES elects one core set for the whole
+// block, so a DES block is never cut. Every step after routing is per row
+// or per token, so the chunked layer computes what the whole one does.
+int host_chunk_plan(const moe_config &c, int64_t bounds[kHostMaxChunks + 1]) {
+  bounds[0] = 0;
+  bounds[1] = c.T;
+  if (c.routing == MOE_DES_VOTE || c.routing == MOE_DES_SEQ) return 1;
+  if (c.T < 2 * kHostMinChunkTokens) return 1;
+  const double act_bytes = (double)c.T * c.d * elem_bytes(c.dtype);
+  const bool two = c.T < 4 * kHostMinChunkTokens ||
+                   layer_weight_bytes(c) > kHostThirdChunkRatio * act_bytes;
+  const int *w = two ? kHostPlan2 : kHostPlan3;
+  const int nw = (int)(two ? sizeof(kHostPlan2) : sizeof(kHostPlan3)) / (int)sizeof(int);
+  const int64_t unit = c.routing == MOE_EXPERT_CHOICE ? c.group_size : 128;
+  int total = 0;
+  for (int i = 0; i < nw; ++i) total += w[i];
+  int n = 0, acc = 0;
+  for (int i = 0; i < nw; ++i) {
+    acc += w[i];
+    int64_t b = i == nw - 1 ? c.T : ((int64_t)c.T * acc / total + unit / 2) / unit * unit;
+    if (b > c.T) b = c.T;
+    if (b > bounds[n]) bounds[++n] = b;
+  }
+  return n;
+}
+
+// The host<->device copies of a token range [t0, t0 + nt).
+struct HostCopy {
+  const uint8_t *xh = nullptr, *rh = nullptr, *zh = nullptr;
+  uint8_t *yh = nullptr;
+  uint8_t *xd = nullptr, *rd = nullptr, *zd = nullptr, *yd = nullptr;
+  size_t row = 0, zrow = 0;  // bytes per token of x / y / residual, of z_prev
+
+  int in(int64_t t0, int64_t nt, cudaStream_t s) const {
+    if (nt <= 0) return MOE_OK;
+    MOE_CUDA_TRY(cudaMemcpyAsync(xd + t0 * row, xh + t0 * row, nt * row, cudaMemcpyHostToDevice, s));
+    if (rh && rd)
+      MOE_CUDA_TRY(cudaMemcpyAsync(rd + t0 * row, rh + t0 * row, nt * row, cudaMemcpyHostToDevice, s));
+    if (zh && zd)
+      MOE_CUDA_TRY(cudaMemcpyAsync(zd + t0 * zrow, zh + t0 * zrow, nt * zrow, cudaMemcpyHostToDevice, s));
+    return MOE_OK;
+  }
+  int out(int64_t t0, int64_t nt, cudaStream_t s) const {
+    if (nt <= 0) return MOE_OK;
+    MOE_CUDA_TRY(cudaMemcpyAsync(yh + t0 * row, yd + t0 * row, nt * row, cudaMemcpyDeviceToHost, s));
+    return MOE_OK;
+  }
+};
+
+// Per-device side streams and events of the pipeline, made on first use
+// and kept for the life of the process; callers hold g_host_pipe_mu from
+// the first event record to the final join, so concurrent callers do not
+// interleave their records and waits on the shared events.
+constexpr int kHostMaxDevices = 64;
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t ev[2 + 2 * kHostMaxChunks] = {};
+};
+std::mutex g_host_pipe_mu;
+HostPipe g_host_pipe[kHostMaxDevices];
+
+int host_pipe(HostPipe **p) {
+  int dev = 0;
+  MOE_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kHostMaxDevices) return MOE_ERR_UNSUPPORTED;
+  HostPipe &hp = g_host_pipe[dev];
+  if (!hp.in) {
+    if (!hp.out) MOE_CUDA_TRY(cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking));
+    for (cudaEvent_t &e : hp.ev)
+      if (!e) MOE_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    MOE_CUDA_TRY(cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking));  // last: marks it ready
+  }
+  *p = &hp;
   return MOE_OK;
 }
 
@@ -587,26 +691,67 @@ int moe_forward_host(const moe_config *cfg, const void *x_host, const void *resi
   const Layout L = layout_of(c);
   void *xd = at<void>(ws, L.x_dev), *yd = at<void>(ws, L.y_dev);
   if ((st = check_forward_ptrs(c, xd, W_r, W1, W2, Ws1, Ws2, const_vecs, yd)) != MOE_OK) return st;
-  const size_t act_bytes = (size_t)c.T * c.d * elem_bytes(c.dtype);
-  if (act_bytes) MOE_CUDA_TRY(cudaMemcpyAsync(xd, x_host, act_bytes, cudaMemcpyHostToDevice, stream));
-  const void *rd = nullptr;
-  if (residual_host == x_host) {
-    rd = xd;
-  } else if (residual_host && act_bytes) {
-    void *r = at<void>(ws, L.res_dev);
-    MOE_CUDA_TRY(cudaMemcpyAsync(r, residual_host, act_bytes, cudaMemcpyHostToDevice, stream));
-    rd = r;
+  HostCopy hc;
+  hc.xh = static_cast<const uint8_t *>(x_host);
+  hc.yh = static_cast<uint8_t *>(y_host);
+  hc.rh = residual_host == x_host ? nullptr : static_cast<const uint8_t *>(residual_host);
+  hc.zh = reinterpret_cast<const uint8_t *>(z_prev_host);
+  hc.xd = static_cast<uint8_t *>(xd);
+  hc.yd = static_cast<uint8_t *>(yd);
+  hc.rd = residual_host == nullptr ? nullptr
+          : residual_host == x_host ? hc.xd : at<uint8_t>(ws, L.res_dev);
+  hc.zd = z_prev_host ? at<uint8_t>(ws, L.zp_dev) : nullptr;
+  hc.row = (size_t)c.d * elem_bytes(c.dtype);
+  hc.zrow = (size_t)c.E * 4;
+
+  int64_t bounds[kHostMaxChunks + 1];
+  const int n = host_chunk_plan(c, bounds);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  MOE_CUDA_TRY(cudaStreamIsCapturing(stream, &cap));
+  bool pipelined = n > 1 && cap == cudaStreamCaptureStatusNone;
+  // Every chunk's routing and MLP buffers must lie below the staging slots.
+  for (int i = 0; pipelined && i < n; ++i) {
+    moe_config ci = c;
+    ci.T = (int32_t)(bounds[i + 1] - bounds[i]);
+    pipelined = layout_of(ci).x_dev <= L.x_dev;
   }
-  const float *zd = nullptr;
-  if (z_prev_host && c.T > 0) {
-    float *z = at<float>(ws, L.zp_dev);
-    MOE_CUDA_TRY(cudaMemcpyAsync(z, z_prev_host, (size_t)c.T * c.E * 4, cudaMemcpyHostToDevice, stream));
-    zd = z;
+  if (!pipelined) {
+    if ((st = hc.in(0, c.T, stream)) != MOE_OK) return st;
+    st = forward_device(c, xd, hc.rd, reinterpret_cast<const float *>(hc.zd), W_r, bias, W1, W2,
+                        Ws1, Ws2, const_vecs, yd, nullptr, dev_status, ws, L, stream);
+    if (st != MOE_OK) return st;
+    return hc.out(0, c.T, stream);
   }
-  st = forward_device(c, xd, rd, zd, W_r, bias, W1, W2, Ws1, Ws2, const_vecs, yd, nullptr,
-                      dev_status, ws, L, stream);
-  if (st != MOE_OK) return st;
-  if (act_bytes) MOE_CUDA_TRY(cudaMemcpyAsync(y_host, yd, act_bytes, cudaMemcpyDeviceToHost, stream));
+
+  // Copy-in on one side stream, copy-out on another, the layer on `stream`,
+  // chunk by chunk: chunk i computes while chunk i+1 comes in and chunk i-1
+  // goes out. The side streams fork from `stream` here and join it at the end.
+  std::lock_guard<std::mutex> lock(g_host_pipe_mu);
+  HostPipe *hp = nullptr;
+  if ((st = host_pipe(&hp)) != MOE_OK) return st;
+  MOE_CUDA_TRY(cudaEventRecord(hp->ev[0], stream));
+  MOE_CUDA_TRY(cudaStreamWaitEvent(hp->in, hp->ev[0], 0));
+  for (int i = 0; i < n; ++i) {
+    const int64_t t0 = bounds[i], nt = bounds[i + 1] - bounds[i];
+    if ((st = hc.in(t0, nt, hp->in)) != MOE_OK) return st;
+    MOE_CUDA_TRY(cudaEventRecord(hp->ev[2 + 2 * i], hp->in));
+  }
+  for (int i = 0; i < n; ++i) {
+    const int64_t t0 = bounds[i], nt = bounds[i + 1] - bounds[i];
+    moe_config ci = c;
+    ci.T = (int32_t)nt;
+    MOE_CUDA_TRY(cudaStreamWaitEvent(stream, hp->ev[2 + 2 * i], 0));
+    st = forward_device(ci, hc.xd + t0 * hc.row, hc.rd ? hc.rd + t0 * hc.row : nullptr,
+                        hc.zd ? reinterpret_cast<const float *>(hc.zd + t0 * hc.zrow) : nullptr,
+                        W_r, bias, W1, W2, Ws1, Ws2, const_vecs, hc.yd + t0 * hc.row, nullptr,
+                        dev_status, ws, layout_of(ci), stream);
+    if (st != MOE_OK) return st;
+    MOE_CUDA_TRY(cudaEventRecord(hp->ev[3 + 2 * i], stream));
+    MOE_CUDA_TRY(cudaStreamWaitEvent(hp->out, hp->ev[3 + 2 * i], 0));
+    if ((st = hc.out(t0, nt, hp->out)) != MOE_OK) return st;
+  }
+  MOE_CUDA_TRY(cudaEventRecord(hp->ev[1], hp->out));
+  MOE_CUDA_TRY(cudaStreamWaitEvent(stream, hp->ev[1], 0));
   return MOE_OK;
 }
 

@@ -253,6 +253,8 @@ EDGE = [
     ("constmix_fp32", "mmoe_constmix", dict(T=200, d=64, h=128, h_shared=64, dtype="f32")),
     ("block_topk_T128", "ditmoe_xl", dict(T=128, d=256, E=16, k=4, h=256, n_shared=0)),
     ("block_des_ragged_d_h", "des_vote", dict(T=40, d=1160, E=32, k=4, h=264, M_core=12)),
+    # router weights over 256 KB: the router K-sliced over the CTAs; ragged last slice
+    ("block_des_sliced_router", "des_vote", dict(T=32, d=4104, E=64, k=8, h=128, M_core=32)),
     # DES-Seq (core = union of local top-k_local): the whole-layer kernel,
     # a core smaller than K (one token: empty slots), the full local
     # budget (= vanilla), and the general path past 128 tokens.
