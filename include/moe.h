@@ -330,8 +330,10 @@ MOE_API int moe_combine(const moe_config *cfg, const void *y_perm,
  * act == MOE_SWIGLU:   y = SiLU(x) = x / (1 + exp(-x)), SwiGLU's gate.
  * MMOE page, "MoE++ expert layer" (heavy experts are standard MLPs). The
  * same device functions run in the GEMM epilogues; erf is evaluated by
- * Abramowitz & Stegun 7.1.26 (absolute error <= 1.5e-7; below 6e-7 as
- * evaluated in fp32, so GELU(x) is within 3e-7 |x| of the exact value).
+ * Abramowitz & Stegun 7.1.26 (absolute error <= 1.5e-7), rearranged so
+ * that GELU(x) = max(x, 0) - 0.5 |x| P(t) exp(-x^2/2) and evaluated two
+ * values at a time on packed fp32x2 arithmetic: GELU(x) is within
+ * 4e-7 max(1, |x|) of the exact value.
  *   x, y [n] fp32 device (y may alias x).
  */
 MOE_API int moe_activation(const float *x, float *y, int64_t n, int act,

@@ -783,7 +783,7 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
               for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * uu[i];
             } else {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+              for (int i = 0; i < 32; i += 2) gelu_erf_x2(v[i], v[i + 1]);
             }
             if (valid) {
               int r = row0 + before;

@@ -126,27 +126,67 @@ __device__ __forceinline__ void store8(float *p, const float (&f)[8]) {
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions (1964),
-// formula 7.1.26: erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5)
-// exp(-x^2), t = 1 / (1 + p x), x >= 0, |error| <= 1.5e-7; odd in x.
-// Evaluated in fp32 the absolute error stays below 6e-7 (the final 1 - ...
-// cancels near 0), i.e. GELU(u) within 3e-7 |u|: far below bf16 rounding
-// and fp32 layer tolerances. Branch-free (one reciprocal, one exponential,
-// five FMAs), so the GEMM epilogues spend few issue slots on it.
-__device__ __forceinline__ float erf_as7126(float x) {
-  const float ax = fabsf(x);
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  poly *= t;
-  const float r = fmaf(-poly, __expf(-ax * ax), 1.0f);
-  return copysignf(r, x);
+// Packed fp32x2 arithmetic (sm_100: two fp32 FMAs per issue slot).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
 }
-// GELU(u) = u * Phi(u) = 0.5 u (1 + erf(u / sqrt 2)), the exact (erf) form.
+__device__ __forceinline__ void f2_unpack(uint64_t r, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_splat(float x) { return f2_pack(x, x); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+// GELU(u) = u Phi(u) = 0.5 u (1 + erf(u / sqrt 2)), the exact (erf) form,
+// two values at a time on packed fp32x2 arithmetic (the GEMM epilogues'
+// issue slots are the scarce resource). erf by Abramowitz & Stegun,
+// Handbook of Mathematical Functions (1964), formula 7.1.26: for a >= 0,
+// erf(a) = 1 - P(t) exp(-a^2), P(t) = a1 t + ... + a5 t^5, t = 1/(1 + p a),
+// |error| <= 1.5e-7. With a = |v|/sqrt 2:
+//   GELU(v) = 0.5 v (1 + sign(v) erf(a)) = max(v, 0) - 0.5 |v| P(t) exp(-v^2/2),
+// with -0.5 folded into P's coefficients, 1/sqrt 2 into p, and
+// exp(-v^2/2) = 2^(v^2 (-0.5 log2 e)); branch-free, no cancellation for
+// v < 0 (one reciprocal and one exponential per value, the rest packed).
+// Evaluated in fp32: |error| <= 4e-7 max(1, |v|), far below bf16 rounding
+// and the fp32 layer tolerance.
+__device__ __forceinline__ void gelu_erf_x2(float &v0, float &v1) {
+  const uint64_t ax = f2_pack(fabsf(v0), fabsf(v1)), v = f2_pack(v0, v1);
+  float d0, d1;
+  f2_unpack(f2_fma(ax, f2_splat(0.23164189f), f2_splat(1.0f)), d0, d1);
+  const uint64_t t = f2_pack(rcp_approx(d0), rcp_approx(d1));
+  uint64_t q = f2_fma(f2_splat(-0.5307027145f), t, f2_splat(0.7265760135f));
+  q = f2_fma(q, t, f2_splat(-0.7107068705f));
+  q = f2_fma(q, t, f2_splat(0.142248368f));
+  q = f2_fma(q, t, f2_splat(-0.127414796f));
+  q = f2_mul(f2_mul(q, t), ax);
+  float s0, s1;
+  f2_unpack(f2_mul(f2_mul(v, v), f2_splat(-0.72134752044f)), s0, s1);
+  const uint64_t e = f2_pack(ex2_approx(s0), ex2_approx(s1));
+  f2_unpack(f2_fma(q, e, f2_pack(fmaxf(v0, 0.f), fmaxf(v1, 0.f))), v0, v1);
+}
 __device__ __forceinline__ float gelu_erf(float v) {
-  return 0.5f * v * (1.0f + erf_as7126(v * 0.70710678118654752440f));
+  float a = v, b = v;
+  gelu_erf_x2(a, b);
+  return a;
 }
 // SiLU(u) = u / (1 + exp(-u)), with the accurate expf (a few ulps at any u).
 __device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.0f + expf(-v)); }

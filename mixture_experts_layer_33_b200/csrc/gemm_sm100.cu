@@ -339,7 +339,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
           for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * u[i];
         } else if (ACT == kActGelu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+          for (int i = 0; i < 32; i += 2) gelu_erf_x2(v[i], v[i + 1]);
         }
         if (valid) store_row32<OUT_F32>(pr, row, col0 + c, v);
       }
@@ -561,7 +561,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
           for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * u[i];
         } else if (ACT == kActGelu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+          for (int i = 0; i < 32; i += 2) gelu_erf_x2(v[i], v[i + 1]);
         }
         if (valid) store_row32<OUT_F32>(pr, row, col0 + c, v);
       }

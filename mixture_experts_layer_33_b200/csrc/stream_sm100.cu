@@ -324,7 +324,7 @@ expert_stream_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
           for (int i = 0; i < 32; ++i) v[i] = silu(v[i]) * u[i];
         } else if (up) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+          for (int i = 0; i < 32; i += 2) gelu_erf_x2(v[i], v[i + 1]);
         }
         if (valid) {
 #pragma unroll

@@ -1,8 +1,11 @@
 """The experts' elementwise activations on the GPU against fp64 references.
 
 GELU is the exact erf form (erf by Abramowitz & Stegun 7.1.26, absolute
-error <= 1.5e-7 for the formula, below 6e-7 as evaluated in fp32, so
-|GELU error| <= 3e-7 |x|); SiLU is x / (1 + exp(-x)).
+error <= 1.5e-7 for the formula, rearranged as max(x, 0) - 0.5|x| P(t)
+exp(-x^2/2) and evaluated on packed fp32x2 arithmetic, two values per
+call: |GELU error| <= 4e-7 max(1, |x|)); SiLU is x / (1 + exp(-x)). The
+inputs have odd and even lengths, so both halves of the packed pair and a
+lone tail element are exercised.
 """
 
 import numpy as np
@@ -32,6 +35,23 @@ def test_gelu_matches_exact_erf_form():
     bound = 0.5 * np.abs(x) * 1e-6 + 4 * np.finfo(np.float32).eps * np.abs(ref) + 1e-30
     assert np.all(np.abs(y - ref) <= bound)
     assert y[-2] == 40.0 and y[-1] == 0.0
+    # Odd length: the last element runs alone in its pair.
+    x, y = _run(moe.GELU_ERF, x64[:-1])
+    ref = x * ndtr(x)
+    bound = 0.5 * np.abs(x) * 1e-6 + 4 * np.finfo(np.float32).eps * np.abs(ref) + 1e-30
+    assert np.all(np.abs(y - ref) <= bound)
+    assert y[-1] == 40.0
+
+
+def test_gelu_in_place():
+    from mixture_experts_layer_33_b200 import moe
+    x64 = np.linspace(-6, 6, 1001)
+    x = torch.tensor(x64, dtype=torch.float32, device="cuda")
+    y = torch.empty_like(x)
+    moe.activation(x, y, moe.GELU_ERF)
+    moe.activation(x, x, moe.GELU_ERF)
+    torch.cuda.synchronize()
+    assert torch.equal(x, y)
 
 
 def test_silu_matches_definition():
