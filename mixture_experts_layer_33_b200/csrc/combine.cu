@@ -9,15 +9,18 @@
 // constant experts return a learned vector; "shared experts": one dense
 // expert is always active (added with weight 1).
 //
-// One warp per (token, 256-feature chunk); each lane owns 8 consecutive
-// features and reads them with 16-byte loads; a token's slot metadata is
-// loaded once, one slot per lane, turned into a source row per slot and
-// broadcast by shuffles; the rows of four slots are loaded before any is
-// summed, so a token's loads overlap instead of queueing one behind the
-// other. Expert outputs arrive in the layer dtype; the sum runs in fp32 in
-// slot order (no atomics, so the output is bitwise deterministic) and is
-// rounded once. `residual` may alias `y` (the forward pass writes
-// x + shared(x) into y first).
+// One warp per token; each lane owns 8 consecutive features of every
+// 256-feature chunk and reads them with 16-byte loads. The token's slot
+// metadata is loaded once, one slot per lane (when its slots fit in a
+// warp), and turned into a source row and weight per slot; the row then
+// goes in passes of up to three chunks, each pass issuing the residual,
+// shared-output and slot-row loads of all its chunks before any sum, so a
+// token costs about one dependent round trip per pass after the metadata.
+// The grid holds only resident blocks. Expert outputs arrive in the layer
+// dtype; the sum runs in fp32 in slot order (no atomics, so the output is
+// bitwise deterministic) and is rounded once. `residual` may alias `y`
+// (the forward pass writes x + shared(x) into y first): each lane reads
+// its own features of a chunk before it writes them.
 #include "common.cuh"
 #include "internal.h"
 
@@ -25,7 +28,8 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kBatch = 4;  // slots whose rows are in flight together
+constexpr int kBatch = 2;  // slots whose rows are in flight together
+constexpr int kPass = 3;   // 256-feature chunks per pass
 
 // 8 consecutive elements held raw until they are summed.
 template <typename T> struct Raw8;
@@ -81,6 +85,59 @@ __device__ __noinline__ float2 const_mix_weights(const T *xr, const T *vrow, int
   return make_float2(e0 / (e0 + e1), e1 / (e0 + e1));
 }
 
+// Slot j of token s, one per lane: its source row (the expert's output
+// row, x_s for an identity expert, the learned vector for a constant
+// expert) and weight, or no row (zero expert, a row the dispatch dropped,
+// an id it flagged). *mix marks a mixed constant expert.
+template <typename T>
+__device__ __forceinline__ void slot_meta(const CombineArgs &a, const KindTable &kinds, bool ec,
+                                          int s, int j, const T *x, const T *cv, const T *yp,
+                                          const T *&src, float &wgt, bool &mix) {
+  src = nullptr;
+  wgt = 0.f;
+  mix = false;
+  const int asg = ec ? a.tok_assign[j] : j;
+  const int e = ec ? (int)((asg / a.C) % a.E) : a.sel[asg];
+  const int row = a.row_of[asg];
+  const float wv = a.w[asg];
+  if (e >= 0 && e < a.E) {
+    const int kind = kinds.kind[e];
+    if (kind == MOE_HEAVY) {
+      if (row >= 0) src = yp + (size_t)row * a.d;
+    } else if (kind == MOE_IDENTITY) {
+      src = x + (size_t)s * a.d;
+    } else if (kind == MOE_CONST) {
+      src = cv + (size_t)kinds.cidx[e] * (a.const_mix ? 3 : 1) * a.d;
+      mix = a.const_mix != 0;
+    }
+    wgt = wv;
+  }
+}
+
+// Slots j0 .. j0+31 of token s (one per lane) with mixed constant experts
+// resolved: the warp forms (a0, a1) = softmax(Wc x_s) for each such slot,
+// which keeps w * a1 on v; w * a0 is added to *x_coef when it is given.
+template <typename T>
+__device__ __forceinline__ void slot_group(const CombineArgs &a, const KindTable &kinds, bool ec,
+                                           int s, int j0, int a1, const T *x, const T *cv,
+                                           const T *yp, const T *&src, float &wgt,
+                                           float *x_coef) {
+  const int lane = threadIdx.x & 31;
+  bool mix = false;
+  src = nullptr;
+  wgt = 0.f;
+  if (j0 + lane < a1) slot_meta(a, kinds, ec, s, j0 + lane, x, cv, yp, src, wgt, mix);
+  for (unsigned mm = __ballot_sync(0xffffffffu, mix); mm; mm &= mm - 1u) {
+    const int j = __ffs(mm) - 1;
+    const T *vrow = reinterpret_cast<const T *>(
+        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), j));
+    const float2 m = const_mix_weights(x + (size_t)s * a.d, vrow, a.d);
+    const float wj = __shfl_sync(0xffffffffu, wgt, j);
+    if (x_coef) *x_coef = fmaf(wj, m.x, *x_coef);
+    if (lane == j) wgt = wj * m.y;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTable kinds) {
   const T *__restrict__ x = static_cast<const T *>(a.x);
@@ -94,103 +151,110 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
   const int nw = (gridDim.x * kThreads) >> 5;
   const bool ec = a.routing == MOE_EXPERT_CHOICE;
   const int chunks = (a.d + 255) / 256;
-  const int64_t items = (int64_t)a.T * chunks;
-  // One warp per (token, 256-feature chunk); each lane owns 8 features.
-  for (int64_t it = gw; it < items; it += nw) {
-    const int s = (int)(it / chunks);
-    const int c0 = (int)(it - (int64_t)s * chunks) * 256 + lane * 8;
-    const bool live = c0 < a.d;
+  for (int s = gw; s < a.T; s += nw) {
     int a0, a1;
     if (ec) { a0 = a.tok_ptr[s]; a1 = a.tok_ptr[s + 1]; }
     else { a0 = s * a.k; a1 = a0 + a.k; }
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    if (live && res) load8(res + (size_t)s * a.d + c0, acc);
-    if (live && ysh) {
-      float t[8];
-      load8(ysh + (size_t)s * a.d + c0, t);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += t[i];
+    const bool one_group = a1 - a0 <= 32;
+    // Slot metadata (and the coefficient of x_s from mixed constant
+    // experts) once per token; a token with more than 32 slots re-reads
+    // its later groups' metadata in each pass.
+    const T *m_src = nullptr;
+    float m_w = 0.f, x_coef = 0.f;
+    if (one_group) {
+      slot_group(a, kinds, ec, s, a0, a1, x, cv, yp, m_src, m_w, &x_coef);
+    } else if (a.const_mix) {
+      for (int j0 = a0; j0 < a1; j0 += 32) {
+        const T *q_src;
+        float q_w;
+        slot_group(a, kinds, ec, s, j0, a1, x, cv, yp, q_src, q_w, &x_coef);
+      }
     }
-    float x_coef = 0.f;  // weight of x_s from mixed constant experts
-    for (int j0 = a0; j0 < a1; j0 += 32) {
-      // Lane j holds slot j0 + j: its weight and the first element of its
-      // source row (the expert's output row, x for an identity expert, the
-      // learned vector for a constant expert), or none (zero expert, a row
-      // the dispatch dropped, or an id it flagged).
-      const T *m_src = nullptr;
-      float m_w = 0.f;
-      bool m_mix = false;
-      if (j0 + lane < a1) {
-        const int asg = ec ? a.tok_assign[j0 + lane] : j0 + lane;
-        const int e = ec ? (int)((asg / a.C) % a.E) : a.sel[asg];
-        const int row = a.row_of[asg];
-        const float wv = a.w[asg];
-        if (e >= 0 && e < a.E) {
-          const int kind = kinds.kind[e];
-          if (kind == MOE_HEAVY) {
-            if (row >= 0) m_src = yp + (size_t)row * a.d;
-          } else if (kind == MOE_IDENTITY) {
-            m_src = x + (size_t)s * a.d;
-          } else if (kind == MOE_CONST) {
-            m_src = cv + (size_t)kinds.cidx[e] * (a.const_mix ? 3 : 1) * a.d;
-            m_mix = a.const_mix != 0;
+    const size_t rb = (size_t)s * a.d;
+    for (int cb = 0; cb < chunks; cb += kPass) {
+      int c0[kPass];
+      bool live[kPass];
+      float acc[kPass][8];
+#pragma unroll
+      for (int q = 0; q < kPass; ++q) {
+        c0[q] = (cb + q) * 256 + lane * 8;
+        live[q] = cb + q < chunks && c0[q] < a.d;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[q][i] = 0.f;
+        if (live[q] && res) load8(res + rb + c0[q], acc[q]);
+        if (live[q] && ysh) {
+          float t[8];
+          load8(ysh + rb + c0[q], t);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[q][i] += t[i];
+        }
+      }
+      for (int j0 = a0; j0 < a1; j0 += 32) {
+        const T *g_src = m_src;
+        float g_w = m_w;
+        if (!one_group) slot_group(a, kinds, ec, s, j0, a1, x, cv, yp, g_src, g_w, nullptr);
+        const int nj = min(32, a1 - j0);
+        for (int jb = 0; jb < nj; jb += kBatch) {
+          Raw8<T> raw[kBatch][kPass];
+          const T *src[kBatch];
+          float wgt[kBatch];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            const int j = (jb + u) & 31;
+            src[u] = reinterpret_cast<const T *>(
+                __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(g_src), j));
+            wgt[u] = __shfl_sync(0xffffffffu, g_w, j);
+            if (jb + u >= nj) src[u] = nullptr;
+#pragma unroll
+            for (int q = 0; q < kPass; ++q)
+              if (src[u] && live[q]) raw[u][q].load(src[u] + c0[q]);
           }
-          m_w = wv;
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+            for (int q = 0; q < kPass; ++q)
+              if (src[u] && live[q]) raw[u][q].fma_into(wgt[u], acc[q]);
         }
       }
-      // Mixed constant experts: the warp forms (a0, a1) = softmax(Wc x_s)
-      // for each such slot; the slot keeps w * a1 on v, and w * a0 joins
-      // the coefficient of x_s, added after the slots.
-      for (unsigned mm = __ballot_sync(0xffffffffu, m_mix); mm; mm &= mm - 1u) {
-        const int j = __ffs(mm) - 1;
-        const T *vrow = reinterpret_cast<const T *>(
-            __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(m_src), j));
-        const float2 mix = const_mix_weights(x + (size_t)s * a.d, vrow, a.d);
-        const float a0 = mix.x, a1 = mix.y;
-        const float wj = __shfl_sync(0xffffffffu, m_w, j);
-        x_coef = fmaf(wj, a0, x_coef);
-        if (lane == j) m_w = wj * a1;
-      }
-      const int nj = min(32, a1 - j0);
-      for (int jb = 0; jb < nj; jb += kBatch) {
-        Raw8<T> raw[kBatch];
-        const T *src[kBatch];
-        float wgt[kBatch];
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          const int j = (jb + u) & 31;
-          src[u] = reinterpret_cast<const T *>(
-              __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(m_src), j));
-          wgt[u] = __shfl_sync(0xffffffffu, m_w, j);
-          if (jb + u >= nj || !live) src[u] = nullptr;
-          if (src[u]) raw[u].load(src[u] + c0);
+      for (int q = 0; q < kPass; ++q) {
+        if (!live[q]) continue;
+        if (x_coef != 0.f) {
+          Raw8<T> xs;
+          xs.load(x + rb + c0[q]);
+          xs.fma_into(x_coef, acc[q]);
         }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u)
-          if (src[u]) raw[u].fma_into(wgt[u], acc);
+        store8(y + rb + c0[q], acc[q]);
       }
     }
-    if (live && x_coef != 0.f) {
-      Raw8<T> xs;
-      xs.load(x + (size_t)s * a.d + c0);
-      xs.fma_into(x_coef, acc);
-    }
-    if (live) store8(y + (size_t)s * a.d + c0, acc);
   }
 }
 
 }  // namespace
 
+// Blocks of `kern` that are resident on one SM (asked once per kernel).
+template <typename K>
+int resident_blocks(K kern, int *cache) {
+  if (*cache == 0) {
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, 0) != cudaSuccess || nb < 1)
+      nb = 1;
+    *cache = nb;
+  }
+  return *cache;
+}
+
 int launch_combine(const CombineArgs &a, const KindTable &kinds, cudaStream_t stream) {
   if (a.T == 0) return MOE_OK;
-  const int64_t items = (int64_t)a.T * ((a.d + 255) / 256);
-  int64_t blocks = (items + (kThreads / 32) - 1) / (kThreads / 32);
-  const int64_t cap = (int64_t)num_sms() * 8;
+  static int nb_bf16 = 0, nb_f32 = 0;
+  const bool bf16 = a.dtype == MOE_BF16;
+  const int nb = bf16 ? resident_blocks(combine_kernel<__nv_bfloat16>, &nb_bf16)
+                      : resident_blocks(combine_kernel<float>, &nb_f32);
+  int64_t blocks = ((int64_t)a.T + (kThreads / 32) - 1) / (kThreads / 32);  // a warp per token
+  const int64_t cap = (int64_t)num_sms() * nb;
   if (blocks > cap) blocks = cap;
   const int grid = (int)blocks;
-  if (a.dtype == MOE_BF16) combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(a, kinds);
+  if (bf16) combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(a, kinds);
   else combine_kernel<float><<<grid, kThreads, 0, stream>>>(a, kinds);
   return last_launch_status();
 }
