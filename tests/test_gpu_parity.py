@@ -314,11 +314,14 @@ def test_deterministic_bytes():
     assert np.array_equal(a["y"].view(np.uint32), b["y"].view(np.uint32))
 
 
-def test_bad_indices_are_flagged_not_faulted():
+@pytest.mark.parametrize("T", [64, 2048], ids=["one_block", "multi_block"])
+def test_bad_indices_are_flagged_not_faulted(T):
     # Host-side fault injection: corrupt expert ids in a selection; the
-    # dispatch kernel's bounds checks flag them and drop those assignments.
+    # dispatch kernel's bounds checks flag them and drop those assignments
+    # (T=64: the one-block dispatch; T=2048: count, scan and scatter over
+    # four blocks), and the kept ones still get stable rows and their x rows.
     m = H.moe()
-    cfg = gen.workload("ditmoe_xl", T=64, d=128, h=256, n_shared=0)
+    cfg = gen.workload("ditmoe_xl", T=T, d=128, h=256, n_shared=0)
     c = m.make_config(cfg)
     na = m.num_assignments(c)
     g = torch.Generator(device="cpu").manual_seed(5)
@@ -332,9 +335,22 @@ def test_bad_indices_are_flagged_not_faulted():
     offsets = torch.empty(c.n_heavy + 1, dtype=torch.int32, device="cuda")
     perm = torch.empty(na, dtype=torch.int32, device="cuda")
     row_of = torch.empty(na, dtype=torch.int32, device="cuda")
-    m.dispatch(c, sel, x, None, offsets, perm, row_of, None, None, status, ws)
+    x_perm = torch.empty(na, cfg["d"], dtype=torch.bfloat16, device="cuda")
+    m.dispatch(c, sel, x, x_perm, offsets, perm, row_of, None, None, status, ws)
     torch.cuda.synchronize()
     assert int(status.item()) & m.DEV_BAD_EXPERT
     ro = row_of.cpu().numpy()
     assert ro[3] == -1 and ro[10] == -1
     assert int(offsets[-1].item()) == na - 2
+    # The kept assignments: stable rows by expert, rows gathered from x.
+    keep = np.ones(na, dtype=bool)
+    keep[[3, 10]] = False
+    s_np = sel.cpu().numpy()
+    a_tok = (np.arange(na) // cfg["k"])[keep]
+    ref_off, ref_perm, ref_row, *_ = oracle.dispatch(a_tok, s_np[keep].astype(np.int64),
+                                                     cfg["E_heavy"], T)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), ref_off)
+    np.testing.assert_array_equal(ro[keep], ref_row)
+    n_rows = int(ref_off[-1])
+    np.testing.assert_array_equal(perm.cpu().numpy()[:n_rows], ref_perm)
+    assert torch.equal(x_perm[:n_rows], x[perm[:n_rows].long()])
