@@ -226,6 +226,9 @@ EDGE = [
     ("single_expert", "ditmoe_xl", dict(T=300, d=128, E=1, k=1, h=256, n_shared=0)),
     ("k_equals_E", "ditmoe_xl", dict(T=130, d=128, E=4, k=4, h=256, n_shared=0)),
     ("E_128", "ditmoe_xl", dict(T=257, d=128, E=128, k=8, h=128, n_shared=0)),
+    # widths off the 256 grid: GEMM1 N = 640 (128-wide tiles, GELU) next to
+    # the shared N = 768, GEMM2 N = 384 (192-wide tiles); ragged tokens
+    ("gemm_off_grid_widths", "ditmoe_xl", dict(T=777, d=384, h=640, h_shared=384)),
     ("all_zero_compute", "mmoe", dict(T=200, d=128, h=256, h_shared=128, zero_compute_logit_bias=60.0)),
     ("ec_full_capacity", "ecdit", dict(T=64, group_size=16, d=128, E=4, h=256, capacity=16)),
     ("ec_whole_batch", "ecdit", dict(T=2048, group_size=2048, d=128, E=8, h=256, capacity=512)),
