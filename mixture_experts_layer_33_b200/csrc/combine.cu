@@ -9,13 +9,15 @@
 // constant experts return a learned vector; "shared experts": one dense
 // expert is always active (added with weight 1).
 //
-// One warp per token; each lane owns 8 consecutive features of every
-// 256-feature chunk and reads them with 16-byte loads. The token's slot
-// metadata is loaded once, one slot per lane (when its slots fit in a
-// warp), and turned into a source row and weight per slot; the row then
-// goes in passes of up to three chunks, each pass issuing the residual,
-// shared-output and slot-row loads of all its chunks before any sum, so a
-// token costs about one dependent round trip per pass after the metadata.
+// One warp per token (or, when there are too few tokens to occupy the
+// GPU that way, per 256-feature chunk of a token); each lane owns 8
+// consecutive features of a chunk and reads them with 16-byte loads. The
+// token's slot metadata is loaded once per item, one slot per lane (when
+// its slots fit in a warp), and turned into a source row and weight per
+// slot; the row then goes in passes of up to three chunks, each pass
+// issuing the residual, shared-output and slot-row loads of all its chunks
+// before any sum, so a token costs about one dependent round trip per pass
+// after the metadata.
 // The grid holds only resident blocks. Expert outputs arrive in the layer
 // dtype; the sum runs in fp32 in slot order (no atomics, so the output is
 // bitwise deterministic) and is rounded once. `residual` may alias `y`
@@ -151,7 +153,15 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
   const int nw = (gridDim.x * kThreads) >> 5;
   const bool ec = a.routing == MOE_EXPERT_CHOICE;
   const int chunks = (a.d + 255) / 256;
-  for (int s = gw; s < a.T; s += nw) {
+  // An item is a whole token (its metadata read once), or with few tokens
+  // one 256-feature chunk of a token, so that every warp has work.
+  const int per_item = a.fine ? 1 : chunks;
+  const int items_per_tok = a.fine ? chunks : 1;
+  const int64_t items = (int64_t)a.T * items_per_tok;
+  for (int64_t it = gw; it < items; it += nw) {
+    const int s = (int)(it / items_per_tok);
+    const int c_begin = (int)(it - (int64_t)s * items_per_tok) * per_item;
+    const int c_end = c_begin + per_item < chunks ? c_begin + per_item : chunks;
     int a0, a1;
     if (ec) { a0 = a.tok_ptr[s]; a1 = a.tok_ptr[s + 1]; }
     else { a0 = s * a.k; a1 = a0 + a.k; }
@@ -171,14 +181,14 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
       }
     }
     const size_t rb = (size_t)s * a.d;
-    for (int cb = 0; cb < chunks; cb += kPass) {
+    for (int cb = c_begin; cb < c_end; cb += kPass) {
       int c0[kPass];
       bool live[kPass];
       float acc[kPass][8];
 #pragma unroll
       for (int q = 0; q < kPass; ++q) {
         c0[q] = (cb + q) * 256 + lane * 8;
-        live[q] = cb + q < chunks && c0[q] < a.d;
+        live[q] = cb + q < c_end && c0[q] < a.d;
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[q][i] = 0.f;
         if (live[q] && res) load8(res + rb + c0[q], acc[q]);
@@ -250,12 +260,19 @@ int launch_combine(const CombineArgs &a, const KindTable &kinds, cudaStream_t st
   const bool bf16 = a.dtype == MOE_BF16;
   const int nb = bf16 ? resident_blocks(combine_kernel<__nv_bfloat16>, &nb_bf16)
                       : resident_blocks(combine_kernel<float>, &nb_f32);
-  int64_t blocks = ((int64_t)a.T + (kThreads / 32) - 1) / (kThreads / 32);  // a warp per token
+  // Whole-token items unless that leaves most resident warps idle.
+  const int64_t warps = (int64_t)num_sms() * nb * (kThreads / 32);
+  const int chunks = (a.d + 255) / 256;
+  const int64_t passes = (chunks + kPass - 1) / kPass;
+  CombineArgs ka = a;
+  ka.fine = (int64_t)a.T * passes < warps ? 1 : 0;
+  const int64_t items = (int64_t)a.T * (ka.fine ? chunks : 1);
+  int64_t blocks = (items + (kThreads / 32) - 1) / (kThreads / 32);  // a warp per item
   const int64_t cap = (int64_t)num_sms() * nb;
   if (blocks > cap) blocks = cap;
   const int grid = (int)blocks;
-  if (bf16) combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(a, kinds);
-  else combine_kernel<float><<<grid, kThreads, 0, stream>>>(a, kinds);
+  if (bf16) combine_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(ka, kinds);
+  else combine_kernel<float><<<grid, kThreads, 0, stream>>>(ka, kinds);
   return last_launch_status();
 }
 

@@ -212,6 +212,7 @@ int launch_activation(const float *x, float *y, int64_t n, int act, cudaStream_t
 struct CombineArgs {
   int routing, T, d, E, k, S, C, dtype;
   int const_mix;  // constant experts mix x and v (const_vecs is [n_const, 3, d])
+  int fine;       // set by launch_combine: one 256-feature chunk per warp item
   const void *y_perm, *y_shared;  // expert outputs, in the layer dtype
   const int32_t *sel;
   const float *w;
