@@ -27,6 +27,11 @@
 // bound), frees its tensor memory and returns.
 #include <string.h>
 
+#include <algorithm>
+#include <functional>
+#include <queue>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_ptx.cuh"
@@ -63,11 +68,63 @@ struct ParamsDev {
 struct Sched {
   int n_entries;
   int total_tiles;
+  int prob_end[2];  // tiles of problem 0 are [0, prob_end[0]), problem 1 [prob_end[0], prob_end[1])
   int tile_start[kMaxEntries + 1];
   int prob[kMaxEntries];
   int group[kMaxEntries];
   int row0[kMaxEntries];
   int row_end[kMaxEntries];
+};
+
+// The tiles one CTA pair runs, in order. Every tile of a problem costs the
+// same (its K blocks), so with two problems of different K a round-robin
+// deal can leave some pairs a whole long tile behind the others, which
+// matters when there are few tiles per pair. Instead the longer problem's
+// tiles are dealt round-robin first, and then each tile of the shorter
+// problem, in order, goes to the pair that becomes free first (list
+// scheduling with known durations, equal free times to the lower id). After
+// the long deal the pairs below r hold one long tile more than the rest, so
+// pair c's m-th short slot starts at a known time and its rank in the
+// merged (start time, pair id) order, which is the short tile it gets, has a
+// closed form. Tiles close in the order still run at about the same time,
+// as with round-robin. Equal K (or one problem) is round-robin over the
+// whole table.
+struct TileSeq {
+  int c, P;
+  int startA, nA, startB, nB;
+  int a, b, r, plo;
+  int j, m;
+
+  __device__ void init(const Sched &s, int kb0, int kb1, int n_probs, int id, int n) {
+    c = id; P = n; j = id; m = 0;
+    const int n0 = s.prob_end[0], n1 = n_probs > 1 ? s.prob_end[1] - s.prob_end[0] : 0;
+    if (n1 == 0 || n0 == 0 || kb0 == kb1) {
+      startA = 0; nA = s.total_tiles; startB = 0; nB = 0; a = b = 1;
+    } else if (kb0 > kb1) {
+      startA = 0; nA = n0; a = kb0; startB = n0; nB = n1; b = kb1;
+    } else {
+      startA = n0; nA = n1; a = kb1; startB = 0; nB = n0; b = kb0;
+    }
+    r = nA % P;
+    plo = P - r;
+  }
+  // Next tile of this pair, or -1.
+  __device__ int next() {
+    if (j < nA) { const int t = startA + j; j += P; return t; }
+    if (nB == 0) return -1;
+    int pos;
+    if (c >= r) {  // free at m*b (relative to the lower load after the long deal)
+      const int t = m * b;
+      const int hi_before = t >= a ? (t - a) / b + 1 : 0;  // slots of the r loaded pairs at times <= t
+      pos = m * plo + (c - r) + r * hi_before;
+    } else {       // free at a + m*b
+      const int t = a + m * b;
+      const int lo_before = (t + b - 1) / b;               // slots of the others at times < t
+      pos = m * r + c + plo * lo_before;
+    }
+    ++m;
+    return pos < nB ? startB + pos : -1;
+  }
 };
 
 __device__ __forceinline__ int find_entry(const Sched &s, int t) {
@@ -225,8 +282,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
         run += __shfl_sync(0xffffffffu, inc, 31);
         ne += min(32, pr.n_groups - g0);
       }
+      if (lane == 0) sched.prob_end[pi] = run;
     }
     if (lane == 0) {
+      if (p.n_probs < 2) sched.prob_end[1] = run;
       sched.n_entries = ne;
       sched.total_tiles = run;
       sched.tile_start[ne] = run;
@@ -361,26 +420,35 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
 }
 
 
-// Two-SM variant: a cluster of 2 CTAs computes one 256 x BN tile with
+// Two-SM variant: a cluster of 2 CTAs computes one 256 x (NH*BN) tile with
 // tcgen05.mma.cta_group::2. Each CTA loads its own 128 rows of A and its
-// own half of the BN rows of B (for SwiGLU: gate rows in rank 0, up rows
-// in rank 1), so each SM moves 2/3 of the operand bytes the 1-SM kernel
-// does per unit of MMA work. Both CTAs' loads complete on the leader's
-// (rank 0) full barrier; the leader's single MMA thread issues the M=256
-// MMAs and releases ring slots and accumulators in both CTAs with one
-// multicast commit; both CTAs' epilogue warps read their own TMEM rows and
-// arrive on the leader's accumulator-empty barrier.
-template <int BN, int ACT, bool OUT_F32, int STAGES>
+// own half of the BN rows of B of each of the NH MMAs (for SwiGLU: gate rows
+// in rank 0, up rows in rank 1), so each SM moves 2/3 (NH = 1) or 1/2
+// (NH = 2) of the operand bytes the 1-SM kernel does per unit of MMA work.
+// With NH = 2 the two MMAs of a k-step share the A tile and fill tensor
+// memory (one accumulator, so the epilogue does not overlap the next tile's
+// MMAs): meant for long K, where a tile's MMAs outlast its epilogue many
+// times over. Both CTAs' loads complete on the leader's (rank 0) full
+// barrier; the leader's single MMA thread issues the M=256 MMAs and
+// releases ring slots and accumulators in both CTAs with one multicast
+// commit; both CTAs' epilogue warps read their own TMEM rows and arrive on
+// the leader's accumulator-empty barrier.
+template <int BN, int ACT, bool OUT_F32, int STAGES, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                          const ParamsDev p) {
+  static_assert(NH == 1 || (NH == 2 && ACT != kActSwiglu), "two MMAs per k-step only without gating");
   constexpr int BMP = 2 * BM;                              // rows per pair tile
-  constexpr int BNO = (ACT == kActSwiglu) ? BN / 2 : BN;   // output columns per tile
+  constexpr int BNO = (ACT == kActSwiglu) ? BN / 2 : BN;   // output columns per MMA
+  constexpr int TNO = NH * BNO;                            // output columns per tile
   constexpr uint32_t A_BYTES = BM * BK * 2;                // this CTA's rows of A
-  constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;          // this CTA's half of B
-  constexpr uint32_t STAGE_TX = 2 * (A_BYTES + B_BYTES);   // both CTAs, counted by the leader
-  constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  constexpr uint32_t B_BYTES = (BN / 2) * BK * 2;          // this CTA's half of one MMA's B
+  constexpr uint32_t STAGE_TX = 2 * (A_BYTES + NH * B_BYTES);  // both CTAs, counted by the leader
+  constexpr int NACC = NH == 1 ? 2 : 1;                    // accumulator buffers
+  constexpr uint32_t ACC_COLS = NH * BN;
+  static_assert(NACC * ACC_COLS <= 512, "accumulators exceed tensor memory");
+  constexpr uint32_t TMEM_COLS = (NACC * ACC_COLS <= 256) ? 256 : 512;
   constexpr uint32_t IDESC = idesc_bf16_f32(BMP, BN);
 
   extern __shared__ uint8_t smem_raw[];
@@ -427,7 +495,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     int run = 0, ne = 0;
     for (int pi = 0; pi < p.n_probs; ++pi) {
       const ProbDev &pr = p.pr[pi];
-      const int ntn = (pr.N + BNO - 1) / BNO;
+      const int ntn = (pr.N + TNO - 1) / TNO;
       for (int g0 = 0; g0 < pr.n_groups; g0 += 32) {
         int g = g0 + lane;
         int lo = 0, hi = 0;
@@ -448,8 +516,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         run += __shfl_sync(0xffffffffu, inc, 31);
         ne += min(32, pr.n_groups - g0);
       }
+      if (lane == 0) sched.prob_end[pi] = run;
     }
     if (lane == 0) {
+      if (p.n_probs < 2) sched.prob_end[1] = run;
       sched.n_entries = ne;
       sched.total_tiles = run;
       sched.tile_start[ne] = run;
@@ -460,7 +530,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
   cluster_sync();  // the peer's barriers exist before any cross-CTA arrival
   tc_fence_after();
   const uint32_t tmem_base = tmem_slot;
-  const int total_tiles = sched.total_tiles;
+  TileSeq seq;  // identical in both CTAs of the pair
+  seq.init(sched, (p.pr[0].K + BK - 1) / BK, (p.pr[1].K + BK - 1) / BK, p.n_probs, pair, npairs);
   const uint32_t leader_full0 = mapa_shared(full0, 0);
   const uint32_t leader_tempty0 = mapa_shared(tempty0, 0);
 
@@ -469,15 +540,15 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     int stage = 0;
     uint32_t phase = 0, armed = 0, armed_parity = 0;
     bool ok = true;
-    for (int t = pair; ok && t < total_tiles; t += npairs) {
+    for (int t = seq.next(); ok && t >= 0; t = seq.next()) {
       const int e = find_entry(sched, t);
       const int pi = sched.prob[e];
       const ProbDev &pr = p.pr[pi];
-      const int ntn = (pr.N + BNO - 1) / BNO;
+      const int ntn = (pr.N + TNO - 1) / TNO;
       const int local = t - sched.tile_start[e];
       const int mt = local / ntn, nt = local - mt * ntn;
       const int a_row = sched.row0[e] + mt * BMP + (int)rank * BM;
-      const int b_row = sched.group[e] * pr.b_rows_per_group + nt * BNO +
+      const int b_row = sched.group[e] * pr.b_rows_per_group + nt * TNO +
                         (int)rank * ((ACT == kActSwiglu) ? pr.N : BN / 2);
       const CUtensorMap *mA = pi ? &tmA1 : &tmA0;
       const CUtensorMap *mB = pi ? &tmB1 : &tmB0;
@@ -487,7 +558,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         if (leader) mbar_arrive_expect_tx(full0 + 8 * stage, STAGE_TX);
         const uint32_t fb = leader_full0 + 8 * stage;
         tma_load_2d_pair(sA + stage * A_BYTES, mA, kb * BK, a_row, fb);
-        tma_load_2d_pair(sB + stage * B_BYTES, mB, kb * BK, b_row, fb);
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+          tma_load_2d_pair(sB + (stage * NH + h) * B_BYTES, mB, kb * BK, b_row + h * BN, fb);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -503,27 +576,29 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int t = pair; ok && t < total_tiles; t += npairs) {
+      for (int t = seq.next(); ok && t >= 0; t = seq.next()) {
         const int e = find_entry(sched, t);
         const int nkb = (p.pr[sched.prob[e]].K + BK - 1) / BK;
         if (!mbar_wait_cluster(tempty0 + 8 * acc, acc_phase ^ 1u, &abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait_cluster(full0 + 8 * stage, phase, &abort_flag, p.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = smem_desc_sw128(sA + stage * A_BYTES);
-          const uint64_t bdesc = smem_desc_sw128(sB + stage * B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_pair(d_tmem, adesc + (uint64_t)(2 * kk), bdesc + (uint64_t)(2 * kk), IDESC,
-                        (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+              tc_mma_pair(d_tmem + (uint32_t)(h * BN), adesc + (uint64_t)(2 * kk),
+                          smem_desc_sw128(sB + (stage * NH + h) * B_BYTES) + (uint64_t)(2 * kk), IDESC,
+                          (kb | kk) != 0 ? 1u : 0u);
           tc_commit_pair(empty0 + 8 * stage, 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit_pair(tfull0 + 8 * acc, 0x3);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
       }
       tc_commit_pair(drain, 0x3);
     }
@@ -534,24 +609,24 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     // ---------------- epilogue (both CTAs, own TMEM rows)
     const int quad = warp & 3;                  // TMEM lanes this warp may read
     const int lrow = quad * 32 + lane;
-    const int c_lo = ((warp - 2) / 4) * (BNO / 2);  // this warp's half of the columns
+    const int c_lo = ((warp - 2) / 4) * (TNO / 2);  // this warp's half of the columns
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = pair; t < total_tiles; t += npairs) {
+    for (int t = seq.next(); t >= 0; t = seq.next()) {
       const int e = find_entry(sched, t);
       const ProbDev &pr = p.pr[sched.prob[e]];
-      const int ntn = (pr.N + BNO - 1) / BNO;
+      const int ntn = (pr.N + TNO - 1) / TNO;
       const int local = t - sched.tile_start[e];
       const int mt = local / ntn, nt = local - mt * ntn;
       const int row = sched.row0[e] + mt * BMP + (int)rank * BM + lrow;
       const bool valid = row < sched.row_end[e];
-      const int col0 = nt * BNO;
+      const int col0 = nt * TNO;
       const bool ready = mbar_wait_cluster(tfull0 + 8 * acc, acc_phase, &abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * ACC_COLS);
 #pragma unroll 1
-      for (int c = c_lo; c < c_lo + BNO / 2; c += 32) {
+      for (int c = c_lo; c < c_lo + TNO / 2; c += 32) {
         float v[32];
         tmem_ld32(taddr + c, v);
         if (ACT == kActSwiglu) {
@@ -568,7 +643,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + 8 * acc);
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
@@ -664,12 +739,12 @@ int run_tc(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t 
   return last_launch_status();
 }
 
-template <int BN, int ACT, bool OUT_F32>
+template <int BN, int ACT, bool OUT_F32, int NH = 1>
 int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t stream) {
-  constexpr uint32_t STAGE_BYTES = (BM + BN / 2) * BK * 2;  // per CTA
+  constexpr uint32_t STAGE_BYTES = (BM + NH * BN / 2) * BK * 2;  // per CTA
   constexpr int S0 = (200 * 1024) / STAGE_BYTES;
   constexpr int STAGES = S0 > 8 ? 8 : S0;
-  constexpr int BNO = (ACT == kActSwiglu) ? BN / 2 : BN;
+  constexpr int BNO = NH * ((ACT == kActSwiglu) ? BN / 2 : BN);  // output columns per tile
   const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES;
 
   CUtensorMap maps[4];
@@ -699,7 +774,7 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
   }
   if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; }
   if (max_tiles == 0) return MOE_OK;
-  auto kern = grouped_gemm_pair_kernel<BN, ACT, OUT_F32, STAGES>;
+  auto kern = grouped_gemm_pair_kernel<BN, ACT, OUT_F32, STAGES, NH>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
@@ -757,12 +832,80 @@ static bool use_pair(const GemmProblem *probs, int n_probs, int bn) {
   return groups > 0 && rows >= 256 * groups;
 }
 
+// Longest-first list-scheduling makespan, in K blocks, of the tiles of (at
+// most two) problems on `workers` CTAs (or CTA pairs): the longer problem's
+// tiles first, then each of the other's to the worker free first -- the
+// order the kernels deal them in.
+static int64_t lpt_makespan(const int64_t *tiles, const int64_t *kb, int n, int workers) {
+  int64_t nA = tiles[0], a = kb[0], nB = n > 1 ? tiles[1] : 0, b = n > 1 ? kb[1] : 0;
+  if (nB > 0 && b > a) { std::swap(nA, nB); std::swap(a, b); }
+  std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> load;
+  const int64_t q = nA / workers, r = nA % workers;
+  for (int w = 0; w < workers; ++w) load.push((q + (w < r ? 1 : 0)) * a);
+  for (int64_t i = 0; i < nB; ++i) {
+    const int64_t l = load.top();
+    load.pop();
+    load.push(l + b);
+  }
+  int64_t mx = 0;
+  while (!load.empty()) { mx = std::max(mx, load.top()); load.pop(); }
+  return mx;
+}
+
+// Estimated tiles of height bm and width tn for a problem: its rows' tiles
+// plus, for grouped rows (group sizes are known only on the device), half a
+// ragged tile per group.
+static int64_t est_tiles(const GemmProblem &q, int bm, int tn) {
+  const int64_t m = (q.a_rows + bm - 1) / bm + (q.offsets ? q.n_groups / 2 : 0);
+  return m * ((q.N + tn - 1) / tn);
+}
+
+// Two MMAs per k-step on a CTA pair (256 x 512 or 256 x 384 tiles) for
+// ungated GEMMs with long K (the down projections): the MMA width per output
+// tile, or 0 to keep the narrow tiles (`bn` wide on one SM, or on a pair when
+// `pair`). Measured on B200, the wide tiles run about 1.25x the MMA work per
+// unit time of the one-SM kernel and about 1.1x that of the narrow pair
+// tiles, but their coarser grain costs more in ragged group ends and in the
+// last wave; they are used when the estimated makespans say so.
+static int pick_wide(const GemmProblem *probs, int n_probs, int act, int bn, bool pair) {
+  if (act != kActNone) return 0;
+  int64_t rows = 0, groups = 0;
+  bool w256 = true, w192 = true;
+  for (int i = 0; i < n_probs; ++i) {
+    if (probs[i].K < 2048) return 0;
+    w256 = w256 && probs[i].N % 512 == 0;
+    w192 = w192 && probs[i].N % 384 == 0;
+    rows += probs[i].a_rows;
+    groups += probs[i].offsets ? probs[i].n_groups : 1;
+  }
+  if (groups == 0 || rows < 256 * groups) return 0;
+  const int wbn = w256 ? 256 : w192 ? 192 : 0;
+  if (wbn == 0) return 0;
+  int64_t tn[2], tw[2], kb[2];
+  for (int i = 0; i < n_probs; ++i) {
+    kb[i] = (probs[i].K + BK - 1) / BK;
+    tn[i] = est_tiles(probs[i], pair ? 2 * BM : BM, bn);
+    tw[i] = est_tiles(probs[i], 2 * BM, 2 * wbn);
+  }
+  const int sms = num_sms();
+  // Time per worker in units of one SM's MMA clocks per K block of a
+  // 128 x 1 tile slice: a narrow tile gives each of its SMs 128 x bn, a
+  // wide one 128 x 2*wbn.
+  const double t_narrow = (double)lpt_makespan(tn, kb, n_probs, pair ? sms / 2 : sms) * bn;
+  const double t_wide = (double)lpt_makespan(tw, kb, n_probs, sms / 2) * 2 * wbn;
+  const double gain = pair ? 1.10 : 1.25;
+  return t_wide < t_narrow * gain ? wbn : 0;
+}
+
 int launch_grouped_gemm_bf16(const GemmProblem *probs, int n_probs, int act, bool out_f32,
                              int32_t *dev_status, cudaStream_t stream) {
   if (n_probs < 1 || n_probs > 2) return MOE_ERR_INVALID_ARG;
   if (out_f32) return MOE_ERR_UNSUPPORTED;  // bf16 layers keep every GEMM output in bf16
   const int bn = pick_bn(probs, n_probs, act);
   const bool pair = use_pair(probs, n_probs, bn);
+  const int wide = pick_wide(probs, n_probs, act, bn, pair);
+  if (wide == 256) return run_tc_pair<256, kActNone, false, 2>(probs, n_probs, dev_status, stream);
+  if (wide == 192) return run_tc_pair<192, kActNone, false, 2>(probs, n_probs, dev_status, stream);
 #define MOE_RUN(BN_, ACT_) \
   return pair ? run_tc_pair<BN_, ACT_, false>(probs, n_probs, dev_status, stream) \
               : run_tc<BN_, ACT_, false>(probs, n_probs, dev_status, stream)

@@ -229,6 +229,12 @@ EDGE = [
     # widths off the 256 grid: GEMM1 N = 640 (128-wide tiles, GELU) next to
     # the shared N = 768, GEMM2 N = 384 (192-wide tiles); ragged tokens
     ("gemm_off_grid_widths", "ditmoe_xl", dict(T=777, d=384, h=640, h_shared=384)),
+    # down projections with K >= 2048 and enough tiles to take the CTA-pair
+    # tiles with two MMAs per k-step: 256 x 384 tiles (N = 768, shared
+    # K = 4096 before routed K = 2048, ragged groups) and 256 x 512 tiles
+    # (N = 1024, expert choice)
+    ("gemm2_pair_two_mma_384", "ditmoe_xl", dict(T=3000, d=768, h=2048, h_shared=2048)),
+    ("gemm2_pair_two_mma_512", "ecdit", dict(T=16 * 128, group_size=128, d=1024, E=8, h=2048, capacity=32)),
     ("all_zero_compute", "mmoe", dict(T=200, d=128, h=256, h_shared=128, zero_compute_logit_bias=60.0)),
     ("ec_full_capacity", "ecdit", dict(T=64, group_size=16, d=128, E=4, h=256, capacity=16)),
     ("ec_whole_batch", "ecdit", dict(T=2048, group_size=2048, d=128, E=8, h=256, capacity=512)),
