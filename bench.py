@@ -71,11 +71,28 @@ def fused_block(cfg):
             and cfg["E"] <= 128 and cfg["k"] <= 32 and cfg["d"] <= 32768)
 
 
+def fused_f32(cfg):
+    """Whether moe_forward runs this layer as one kernel with a CTA per token
+    (the library's rule for small fp32 layers: token choice, no shared
+    expert, no mixed constant experts, at most 1024 tokens, k <= 32,
+    d <= 1024 and h <= 2048, both multiples of 4)."""
+    return (cfg["dtype"] == "f32" and cfg["routing"] == "token_topk" and cfg["n_shared"] == 0
+            and not cfg.get("const_mix", 0) and 1 <= cfg["T"] <= 1024 and cfg["E"] <= 128
+            and 1 <= cfg["k"] <= min(32, cfg["E"]) and 4 <= cfg["d"] <= 1024 and cfg["d"] % 4 == 0
+            and 4 <= cfg["h"] <= 2048 and cfg["h"] % 4 == 0)
+
+
+# fp32 FMA lanes per SM on B200 (4 SM sub-partitions x 32): the peak of the
+# CUDA-core fp32 path is 148 SMs x 128 lanes x 2 FLOP per clock.
+FP32_LANES_PER_SM = 128
+
+
 def forward_launches(cfg):
     """Kernels one moe_forward launches for this workload (the library's
-    path choice: fused small block; split router + fused routing for other
-    blocks of <= 128 tokens; split router for <= 512; else the full router)."""
-    if fused_block(cfg):
+    path choice: one kernel for small fp32 layers and for small bf16 blocks;
+    split router + fused routing for other blocks of <= 128 tokens; split
+    router for <= 512; else the full router)."""
+    if fused_block(cfg) or fused_f32(cfg):
         return 1
     bf16 = cfg["dtype"] == "bf16"
     r = cfg["routing"]
@@ -441,7 +458,7 @@ def gpu_bench(args):
     # events around it; its one kernel (after a memset of its sync words) is
     # the dominant launch, so this bounds that kernel's duration from above.
     fused_ms = None
-    if fused_block(cfg):
+    if fused_block(cfg) or fused_f32(cfg):
         fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
         torch.cuda.synchronize()
@@ -484,7 +501,17 @@ def gpu_bench(args):
     tr = NCU_TRAFFIC.get(cfg["name"])
     traffic = tr["bytes"] if tr and tr["sha256_16"] == source_hash(tr["source"]) else None
     gm_ms = stage_ms["grouped_mlp"] / args.steps  # grouped-MLP launches, from timed region 2
-    if cfg["dtype"] == "bf16" and cfg["T"] <= 128:  # small blocks stream expert weights
+    if fused_f32(cfg) and fused_ms is not None:
+        # One kernel on CUDA cores: fp32 FMAs against the fp32 lanes' peak at
+        # the maximum SM clock (latency-bound at these sizes).
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        pk = sms * FP32_LANES_PER_SM * 2 * clocks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        achieved = flops / (fused_ms / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": "small_f32_kernel (whole layer, one launch after a memset)",
+                "achieved": round(achieved, 2), "peak": round(pk, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / pk, 4), "traffic": None, "algorithmic_per_launch": flops,
+                "peak_source": f"derived: {sms} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 FLOP x max SM clock"}
+    elif cfg["dtype"] == "bf16" and cfg["T"] <= 128:  # small blocks stream expert weights
         bytes_ = weight_bytes_used(cfg, used)
         if fused_ms is not None:
             kname = "moe_block_kernel (whole layer, one launch after a memset)"

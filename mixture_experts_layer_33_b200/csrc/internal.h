@@ -123,6 +123,23 @@ void block_zero_layout(BlockArgs &a, void *z, int E);
 int launch_moe_block(const BlockArgs &a, const KindTable &kinds, const void *W1, const void *W2,
                      int act, cudaStream_t stream);
 
+// small_f32.cu: the whole layer for a small fp32 token-choice layer without
+// a shared expert, one CTA per token (router row, softmax, top-k, the
+// experts' MLPs from L2-resident weights, combine), one launch. `counts`
+// (small_f32_zero_bytes: one word per heavy expert, then a CTA counter)
+// must be zero at launch.
+struct SmallF32Args {
+  const float *x, *residual, *W_r, *bias, *zprev, *W1, *W2, *const_vecs;
+  float zscale;
+  int T, d, h, E, n_heavy, k, renorm, gated;
+  float *logits, *probs, *w, *y;
+  int32_t *sel, *offsets;
+  unsigned *counts;
+};
+bool small_f32_supported(const moe_config &c);
+size_t small_f32_zero_bytes(int n_heavy);
+int launch_small_f32(const SmallF32Args &a, const KindTable &kinds, cudaStream_t stream);
+
 int launch_select_topk(const float *logits, const float *probs, int T, int E,
                        int k, int renorm, int32_t *idx, float *w,
                        cudaStream_t stream);

@@ -89,7 +89,8 @@ int n_const_of(const moe_config &c) {
 // Workspace layout shared by the entry points.
 struct Layout {
   size_t logits, probs, sel, w, votes, core, offsets, perm, row_of, tok_ptr, tok_assign, dpart,
-      x_perm, H, H_sh, Y, Y_sh, done, rpart, bzero, cbar, x_dev, res_dev, zp_dev, y_dev, total;
+      x_perm, H, H_sh, Y, Y_sh, done, rpart, bzero, fzero, cbar, x_dev, res_dev, zp_dev, y_dev,
+      total;
 };
 
 Layout layout_of(const moe_config &c) {
@@ -125,6 +126,7 @@ Layout layout_of(const moe_config &c) {
     L.rpart = take((size_t)(parts > slices ? parts : slices) * c.T * c.E * 4);
   }
   L.bzero = take(moe_block_supported(c) ? block_zero_bytes(c.E, c.n_heavy) : 0);
+  L.fzero = take(small_f32_supported(c) ? small_f32_zero_bytes(c.n_heavy) : 0);
   // Small-block routing kernel: grid-barrier counter (16 B), then a 4-word
   // token bitmask per expert.
   L.cbar = take(16 + (size_t)c.E * 16);
@@ -370,6 +372,24 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
   const int n_part = router_split_parts(c.T, c.d, c.dtype);
   const bool streaming = c.dtype == MOE_BF16 && stream_mlp_supported(c.T);
   bool routed_and_gathered = false;
+  if (small_f32_supported(c)) {
+    // Small fp32 token-choice layer without a shared expert: the whole layer
+    // in one launch, a CTA per token (its per-expert row counts, and the
+    // CTA counter that finds the last CTA, start at zero).
+    MOE_CUDA_TRY(cudaMemsetAsync(at<void>(ws, L.fzero), 0, small_f32_zero_bytes(c.n_heavy), stream));
+    SmallF32Args fa{};
+    fa.x = static_cast<const float *>(x);
+    fa.residual = static_cast<const float *>(residual);
+    fa.W_r = static_cast<const float *>(W_r);
+    fa.bias = bias; fa.zprev = z_prev; fa.zscale = c.gate_residual_scale;
+    fa.W1 = static_cast<const float *>(W1); fa.W2 = static_cast<const float *>(W2);
+    fa.const_vecs = static_cast<const float *>(const_vecs);
+    fa.T = c.T; fa.d = c.d; fa.h = c.h; fa.E = c.E; fa.n_heavy = c.n_heavy; fa.k = c.k;
+    fa.renorm = c.renorm; fa.gated = c.act == MOE_SWIGLU;
+    fa.logits = logits; fa.probs = probs; fa.w = w; fa.y = static_cast<float *>(y);
+    fa.sel = sel; fa.offsets = offsets; fa.counts = at<unsigned>(ws, L.fzero);
+    return launch_small_f32(fa, kind_table(c), stream);
+  }
   if (moe_block_supported(c)) {
     // Small bf16 block without a shared expert: the whole layer in one
     // persistent kernel (router K-sliced over the CTAs, selection, a weight

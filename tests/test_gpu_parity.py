@@ -244,6 +244,14 @@ EDGE = [
     ("des_beta_one", "des_vote", dict(d=128, h=128, M_core=64)),
     ("odd_N_swiglu_routed", "des_vote", dict(T=37, d=128, E=16, k=4, h=128, M_core=8)),
     ("tiny_fp32_k1", "tiny_fp32", dict(k=1)),
+    # fp32 token-choice layers of <= 1024 tokens without a shared expert run
+    # as one launch (a CTA per token): zero-computation experts, gate
+    # residual and SwiGLU; renormalised weights over 16 experts; one token.
+    # Past 1024 tokens the general fp32 path (dispatch, grouped GEMMs).
+    ("f32_one_launch_kinds_swiglu", "mmoe", dict(T=200, d=64, h=128, n_shared=0, dtype="f32", act="swiglu")),
+    ("f32_one_launch_renorm_E16", "ditmoe_xl", dict(T=300, d=96, E=16, k=4, h=160, n_shared=0, dtype="f32", renorm=1)),
+    ("f32_one_launch_one_token", "tiny_fp32", dict(T=1)),
+    ("f32_general_path_T2048", "tiny_fp32", dict(T=2048)),
     # Blocks of <= 128 tokens route, dispatch and gather in one cooperative
     # kernel; 129 tokens take the separate finish / dispatch / gather kernels.
     ("small_block_T128_mmoe", "mmoe", dict(T=128, d=128, h=256, h_shared=128)),
