@@ -242,24 +242,23 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
 
 }  // namespace
 
-// Blocks of `kern` that are resident on one SM (asked once per kernel).
+// Blocks of `kern` that are resident on one SM.
 template <typename K>
-int resident_blocks(K kern, int *cache) {
-  if (*cache == 0) {
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, 0) != cudaSuccess || nb < 1)
-      nb = 1;
-    *cache = nb;
-  }
-  return *cache;
+int resident_blocks(K kern) {
+  int nb = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, 0) != cudaSuccess || nb < 1)
+    nb = 1;
+  return nb;
 }
 
 int launch_combine(const CombineArgs &a, const KindTable &kinds, cudaStream_t stream) {
   if (a.T == 0) return MOE_OK;
-  static int nb_bf16 = 0, nb_f32 = 0;
+  // Asked once per kernel (function-local statics are initialised once,
+  // safely under concurrent first calls).
+  static const int nb_bf16 = resident_blocks(combine_kernel<__nv_bfloat16>);
+  static const int nb_f32 = resident_blocks(combine_kernel<float>);
   const bool bf16 = a.dtype == MOE_BF16;
-  const int nb = bf16 ? resident_blocks(combine_kernel<__nv_bfloat16>, &nb_bf16)
-                      : resident_blocks(combine_kernel<float>, &nb_f32);
+  const int nb = bf16 ? nb_bf16 : nb_f32;
   // Whole-token items unless that leaves most resident warps idle.
   const int64_t warps = (int64_t)num_sms() * nb * (kThreads / 32);
   const int chunks = (a.d + 255) / 256;
