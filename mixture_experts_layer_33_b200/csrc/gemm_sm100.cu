@@ -790,9 +790,16 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.gridDim = dim3(2 * (unsigned)(num_sms() / 2));
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1)
-    return MOE_ERR_UNSUPPORTED;
+  // Co-resident CTA pairs of this kernel, asked once per instantiation (a
+  // function-local static is initialised once, safely under concurrent
+  // first calls).
+  static const int max_clusters = [&] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    return n;
+  }();
+  int clusters = max_clusters;
+  if (clusters < 1) return MOE_ERR_UNSUPPORTED;
   if (max_tiles < clusters) clusters = (int)max_tiles;
   cfg.gridDim = dim3(2 * (unsigned)clusters);
   MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], pd));
@@ -840,6 +847,11 @@ static bool use_pair(const GemmProblem *probs, int n_probs, int bn) {
 static int64_t lpt_makespan(const int64_t *tiles, const int64_t *kb, int n, int workers) {
   int64_t nA = tiles[0], a = kb[0], nB = n > 1 ? tiles[1] : 0, b = n > 1 ? kb[1] : 0;
   if (nB > 0 && b > a) { std::swap(nA, nB); std::swap(a, b); }
+  // With many tiles per worker the last wave is a small part of the whole:
+  // the mean load plus one long tile bounds the makespan without simulating
+  // every tile (this runs on the host at every launch).
+  if (nA + nB > 32 * (int64_t)workers)
+    return (nA * a + nB * b + workers - 1) / workers + a;
   std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> load;
   const int64_t q = nA / workers, r = nA % workers;
   for (int w = 0; w < workers; ++w) load.push((q + (w < r ? 1 : 0)) * a);
