@@ -59,6 +59,10 @@ NCU_TRAFFIC = {
                  "source": "block_sm100.cu", "sha256_16": "9d32a6811d13f0ac"},
     "ditmoe_xl": {"bytes": (162.94 + 258.17 + 459.52 + 38.40) * 1e6,
                   "source": "gemm_sm100.cu", "sha256_16": "cfc640b5c5107701"},
+    "ecdit": {"bytes": (1256.95 + 252.12 + 1474.95 + 58.29) * 1e6,
+              "source": "gemm_sm100.cu", "sha256_16": "cfc640b5c5107701"},
+    "mmoe": {"bytes": (231.67 + 155.34 + 421.20 + 40.03) * 1e6,
+             "source": "gemm_sm100.cu", "sha256_16": "cfc640b5c5107701"},
 }
 
 
