@@ -28,6 +28,8 @@ CASES = [
     ("des_vote", {}, False),
     # below two minimum chunks: one chunk
     ("ditmoe_xl", dict(T=3000, d=256, h=512, h_shared=256), True),
+    # a small fp32 layer: one chunk, the one-launch fp32 path
+    ("tiny_fp32", {}, True),
 ]
 
 
