@@ -206,6 +206,78 @@ __global__ void __launch_bounds__(kThreads) token_csr_kernel(DispatchArgs a) {
   }
 }
 
+// Expert choice in one launch, one CTA per routing group. EC-DiT, section
+// 3 (Expert-Choice routing): every expert takes exactly C tokens of every
+// group, so the stable permutation by (expert, token) has a closed form:
+// expert e's rows start at e*G*C, and the c-th token (ascending) that
+// expert took from group g lands in row e*G*C + g*C + c (groups are
+// consecutive token ranges, so rows stay in ascending token order within
+// an expert). No histogram, scan or scatter; the group's token ids are
+// staged in shared memory once, and the per-token assignment lists (in
+// expert order, for the combine) are built from there.
+__global__ void __launch_bounds__(kThreads) dispatch_ec_kernel(DispatchArgs a) {
+  extern __shared__ int sm[];
+  const int S = a.S, E = a.E, C = a.C, G = gridDim.x, g = blockIdx.x;
+  int *cnt = sm;        // [S]
+  int *ptr = sm + S;    // [S]
+  int *tk = sm + 2 * S; // [E * C] token (within the group) of each assignment, or -1
+  __shared__ int scratch[33];
+  clear_words(a);
+  const int64_t abase = (int64_t)g * E * C;
+  const int64_t per_expert = (int64_t)G * C;
+  if (g == 0)
+    for (int e = threadIdx.x; e <= a.n_heavy; e += kThreads) a.offsets[e] = (int32_t)(e * per_expert);
+  for (int t = threadIdx.x; t < S; t += kThreads) cnt[t] = 0;
+  __syncthreads();
+  for (int j = threadIdx.x; j < E * C; j += kThreads) {
+    const int e = j / C, c = j - (j / C) * C;
+    int t = a.sel[abase + j] - g * S;
+    if (t < 0 || t >= S) {
+      set_status(a.dev_status, MOE_DEV_BAD_TOKEN);
+      t = -1;
+    } else {
+      atomicAdd(&cnt[t], 1);
+    }
+    tk[j] = t;
+    if (e < a.n_heavy) {
+      const int64_t row = e * per_expert + (int64_t)g * C + c;
+      // A dropped token still owns its row (the layout is fixed): it
+      // gathers the group's first token and no slot reads its output.
+      a.perm[row] = g * S + (t >= 0 ? t : 0);
+      a.row_of[abase + j] = t >= 0 ? (int32_t)row : -1;
+    } else {
+      a.row_of[abase + j] = -1;
+    }
+  }
+  __syncthreads();
+  if (a.tok_ptr && a.tok_assign) {
+    const int per = (S + kThreads - 1) / kThreads;
+    const int lo = threadIdx.x * per, hi = min(S, lo + per);
+    int mine = 0;
+    for (int t = lo; t < hi; ++t) mine += cnt[t];
+    int total;
+    int run = block_exclusive_scan(mine, scratch, &total);
+    for (int t = lo; t < hi; ++t) {
+      ptr[t] = run;
+      a.tok_ptr[(size_t)g * S + t] = (int32_t)(abase + run);
+      run += cnt[t];
+      cnt[t] = 0;  // reused as the fill count
+    }
+    if (g == G - 1 && threadIdx.x == 0) a.tok_ptr[(size_t)G * S] = (int32_t)(abase + total);
+    __syncthreads();
+    for (int e = 0; e < E; ++e) {  // expert order: one expert's tokens are distinct
+      for (int c = threadIdx.x; c < C; c += kThreads) {
+        const int t = tk[e * C + c];
+        if (t >= 0) {
+          const int slot = atomicAdd(&cnt[t], 1);
+          a.tok_assign[abase + ptr[t] + slot] = (int32_t)(abase + (int64_t)e * C + c);
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // x_perm[r] = x[perm[r]] for r < offsets[n_heavy], 16-byte vectors.
 __global__ void __launch_bounds__(kThreads)
 gather_rows_kernel(const uint4 *__restrict__ x, uint4 *__restrict__ xp, const int32_t *__restrict__ perm,
@@ -251,6 +323,28 @@ int launch_dispatch(const DispatchArgs &a, void *ws, cudaStream_t stream) {
     st = last_launch_status();
   }
   return st;
+}
+
+// Shared memory of dispatch_ec_kernel: two words per token of a group and
+// one per assignment of a group.
+static size_t dispatch_ec_smem(int S, int E, int C) {
+  return (2 * (size_t)S + (size_t)E * C) * sizeof(int);
+}
+
+bool dispatch_ec_supported(int S, int E, int C) {
+  return S >= 1 && C >= 1 && dispatch_ec_smem(S, E, C) <= 48 * 1024;
+}
+
+int launch_dispatch_ec(const DispatchArgs &a, cudaStream_t stream) {
+  if (a.T == 0 || a.S < 1) {
+    MOE_CUDA_TRY(cudaMemsetAsync(a.offsets, 0, (a.n_heavy + 1) * sizeof(int32_t), stream));
+    if (a.n_zero_words > 0)
+      MOE_CUDA_TRY(cudaMemsetAsync(a.zero_words, 0, a.n_zero_words * sizeof(int32_t), stream));
+    if (a.tok_ptr) MOE_CUDA_TRY(cudaMemsetAsync(a.tok_ptr, 0, sizeof(int32_t), stream));
+    return MOE_OK;
+  }
+  dispatch_ec_kernel<<<a.T / a.S, kThreads, dispatch_ec_smem(a.S, a.E, a.C), stream>>>(a);
+  return last_launch_status();
 }
 
 int launch_gather_rows(const void *x, void *x_perm, const int32_t *perm, const int32_t *offsets,

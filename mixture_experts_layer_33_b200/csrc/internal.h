@@ -173,6 +173,10 @@ struct DispatchArgs {
 };
 size_t dispatch_workspace_bytes(int64_t n_assign, int n_heavy);
 int launch_dispatch(const DispatchArgs &a, void *ws, cudaStream_t stream);
+// Expert choice in one launch (the permutation in closed form, one CTA per
+// routing group) for groups whose token ids fit in shared memory.
+bool dispatch_ec_supported(int S, int E, int C);
+int launch_dispatch_ec(const DispatchArgs &a, cudaStream_t stream);
 // dispatch_noalloc.cu: the dispatch with library-owned scratch.
 bool dispatch_fits_noalloc_scratch(int64_t n_assign, int n_heavy);
 int launch_dispatch_noalloc(const DispatchArgs &a, cudaStream_t stream);

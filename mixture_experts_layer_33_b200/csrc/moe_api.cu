@@ -474,7 +474,12 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
       da.zero_words = at<int32_t>(ws, L.done);
       da.n_zero_words = c.n_heavy + 1;
     }
-    st = launch_dispatch(da, at<void>(ws, L.dpart), stream);
+    // The selection above is this library's own: under expert choice every
+    // token id is in its group and every expert has exactly C of them.
+    if (c.routing == MOE_EXPERT_CHOICE && dispatch_ec_supported(c.group_size, c.E, c.capacity))
+      st = launch_dispatch_ec(da, stream);
+    else
+      st = launch_dispatch(da, at<void>(ws, L.dpart), stream);
     if (st != MOE_OK) return st;
     if (c.n_heavy > 0) {
       st = launch_gather_rows(x, x_perm, perm, offsets, c.n_heavy, na, c.d, elem_bytes(c.dtype), stream);
