@@ -36,7 +36,11 @@ constexpr int kThreads = 128;
 constexpr int kRowwiseMaxTokens = 512;  // bf16 layers this small use one CTA per token
 constexpr int kMmaBM = 32;               // tokens per CTA of the MMA router (2 warps x 16)
 constexpr int kMmaThreads = 64;
-constexpr int kMmaStages = 6;            // cp.async ring depth: many x tiles in flight per SM
+// cp.async ring depth: with up to 32 experts twelve 64-wide slices of the
+// token tile are in flight per CTA (a 1152-wide tile in 1.5 round trips);
+// wider expert tiles keep six to stay within shared memory.
+template <int NT>
+constexpr int mma_stages() { return NT <= 4 ? 12 : 6; }
 
 // Softmax of one token row held by a warp: expert e = lane + 32*v.
 template <int VPL>
@@ -103,6 +107,7 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
                    ZeroList zero) {
   constexpr int EP = NT * 8;
   constexpr int VPL = (EP + 31) / 32;
+  constexpr int kMmaStages = mma_stages<NT>();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16 *sX = reinterpret_cast<__nv_bfloat16 *>(smem_raw);   // [stages][kMmaBM][kLDS]
   __nv_bfloat16 *sW = sX + kMmaStages * kMmaBM * kLDS;                      // [stages][EP][kLDS]
@@ -494,6 +499,7 @@ int run_router_bf16(const void *x, const void *Wr, const float *bias, const floa
                     float zscale, int T, int d, int E, float *logits, float *probs, int k,
                     int renorm, int32_t *idx, float *w, cudaStream_t stream) {
   constexpr int EP = NT * 8;
+  constexpr int kMmaStages = mma_stages<NT>();
   const size_t smem = (size_t)kMmaStages * (kMmaBM + EP) * kLDS * sizeof(__nv_bfloat16) +
                       (size_t)kMmaBM * (EP + 1) * sizeof(float);
   auto kern = router_bf16_kernel<NT>;
@@ -509,6 +515,7 @@ template <int NT>
 int run_router_partial(const void *x, const void *Wr, int T, int d, int E, float *part,
                        int n_part, const ZeroList &zero, cudaStream_t stream) {
   constexpr int EP = NT * 8;
+  constexpr int kMmaStages = mma_stages<NT>();
   const size_t smem = (size_t)kMmaStages * (kMmaBM + EP) * kLDS * sizeof(__nv_bfloat16) +
                       (size_t)kMmaBM * (EP + 1) * sizeof(float);
   auto kern = router_bf16_kernel<NT, true>;
