@@ -63,6 +63,8 @@ constexpr int kMaxK = 32;
 constexpr int BMW = 128;  // weight rows per unit (MMA M)
 constexpr int BK = 64;
 constexpr int kUQ = 8;  // unit-id ring between the producer and the other roles
+// Bytes of leading weight boxes warmed into L2 while the routing runs.
+constexpr int64_t kWarmBytes = 32ll << 20;
 
 __device__ __forceinline__ void epi_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
@@ -144,6 +146,38 @@ __device__ __forceinline__ void fma8(float wgt, const uint4 &u, float (&acc)[8])
     acc[2 * i] = fmaf(wgt, f.x, acc[2 * i]);
     acc[2 * i + 1] = fmaf(wgt, f.y, acc[2 * i + 1]);
   }
+}
+
+// Unit u of the grid-wide list. Up units come first: block 0 of every
+// streamed expert (the blocks whose leading weight boxes were warmed into
+// L2 during the routing), then the other blocks expert by expert; then the
+// down units expert by expert. gi indexes the streamed-expert list.
+struct BlockUnit {
+  bool up;
+  int gi, blk;
+};
+__device__ __forceinline__ BlockUnit unit_of(int u, int n_groups, int up_blocks, int down_blocks) {
+  BlockUnit r;
+  const int n_up = n_groups * up_blocks;
+  r.up = u < n_up;
+  if (!r.up) {
+    r.gi = (u - n_up) / down_blocks;
+    r.blk = (u - n_up) % down_blocks;
+  } else if (u < n_groups) {
+    r.gi = u;
+    r.blk = 0;
+  } else {  // up_blocks >= 2 here
+    r.gi = (u - n_groups) / (up_blocks - 1);
+    r.blk = 1 + (u - n_groups) % (up_blocks - 1);
+  }
+  return r;
+}
+
+__device__ __forceinline__ void prefetch_box_l2(const CUtensorMap *map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 template <int NB, int ACT>
@@ -315,6 +349,23 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
     ok_slot = wait_u32(a.sync + 0, (unsigned)G, &abort_flag, a.dev_status) ? 1 : 0;
   }
   __syncthreads();
+
+  // CTAs without a token warm L2 with the leading k-blocks of block 0 of
+  // every heavy expert's up projection (up to kWarmBytes): which experts
+  // will stream is not known until the votes are in, HBM is idle until
+  // then, and block 0 of each streamed expert is the first unit claimed.
+  if (t >= T && ok_slot && tid == 0 && nh > 0) {
+    const int per = GATED ? 2 : 1;  // gate and up rows
+    const int nkb = (a.d + BK - 1) / BK;
+    const int64_t fit = kWarmBytes / ((int64_t)nh * per * BMW * BK * 2);
+    const int pk = (int)(fit < nkb ? fit : nkb);
+    const int n_box = nh * per * pk;
+    for (int i = t - T; i < n_box; i += G - T) {
+      const int e = i / (per * pk), r = i - e * (per * pk);
+      const int half = r / pk, kb = r - half * pk;
+      prefetch_box_l2(&tmW1, kb * BK, e * a.w1_rows_per_group + half * a.h);
+    }
+  }
 
   // ---- 1. token CTAs finish the router and pick.
   if (t < T && ok_slot) {
@@ -527,7 +578,7 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
           __threadfence_block();  // the offsets written before the flag
           // The routing is known: an expert that got no rows needs no
           // weights (the unit is passed on as skipped: -2 - u).
-          const int g0 = u < n_up ? glist[u / up_blocks] : glist[(u - n_up) / down_blocks];
+          const int g0 = glist[unit_of(u, n_groups, up_blocks, down_blocks).gi];
           if (offs[g0 + 1] == offs[g0]) code = -2 - u;
         }
         if (!mbar_wait(uqe0 + 8 * qs, qph ^ 1u, &abort_flag, a.dev_status)) { ok = false; break; }
@@ -536,9 +587,10 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
         if (++qs == kUQ) { qs = 0; qph ^= 1u; }
         if (u < 0) break;
         if (code < -1) continue;
-        const bool up = u < n_up;
-        const int g = up ? glist[u / up_blocks] : glist[(u - n_up) / down_blocks];
-        const int blk = up ? u % up_blocks : (u - n_up) % down_blocks;
+        const BlockUnit un = unit_of(u, n_groups, up_blocks, down_blocks);
+        const bool up = un.up;
+        const int g = glist[un.gi];
+        const int blk = un.blk;
         const CUtensorMap *mW = up ? &tmW1 : &tmW2;
         const CUtensorMap *mB = up ? &tmX : &tmH;
         const int w_row = up ? g * w1_rows + blk * BMW : g * down_N + blk * BMW;
@@ -749,15 +801,16 @@ moe_block_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_constant
         const int su = -2 - code;
         __syncwarp();
         if (lane == 0) {
-          if (su < n_up) atomicAdd(a.done + glist[su / up_blocks], 1);
+          if (su < n_up) atomicAdd(a.done + glist[unit_of(su, n_groups, up_blocks, down_blocks).gi], 1);
           mbar_arrive(uq_done);
         }
         continue;
       }
       const int u = code;
-      const bool up = u < n_up;
-      const int g = up ? glist[u / up_blocks] : glist[(u - n_up) / down_blocks];
-      const int blk = up ? u % up_blocks : (u - n_up) % down_blocks;
+      const BlockUnit un = unit_of(u, n_groups, up_blocks, down_blocks);
+      const bool up = un.up;
+      const int g = glist[un.gi];
+      const int blk = un.blk;
       const int N = up ? up_N : down_N;
       const int feat = blk * BMW + quad * 32 + lane;
       const bool valid = feat < N;
