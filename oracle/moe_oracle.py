@@ -395,11 +395,14 @@ def heavy_expert(act, X, W1e, W2e, h):
 # experts": always active; reading R17 for the residual).
 # --------------------------------------------------------------------------
 def combine(tokens, a_tok, a_exp, a_w, expert_out, residual=None,
-            shared_out=None):
+            shared_out=None, d=None):
     """y_s = r_s + shared(x_s) + sum over the assignments a of s of w_a * E_{e_a}(x_s).
 
     ``expert_out(a)`` returns the [d] output of assignment a's expert on
-    its token. Returns y for the requested ``tokens`` (in that order).
+    its token. Returns y for the requested ``tokens`` (in that order). A
+    token with no residual, no shared output and no expert (expert choice
+    can leave a token unpicked) sums nothing: its row is 0, which needs the
+    model width ``d`` when no other row shows it.
     """
     tokens = np.asarray(tokens, dtype=np.int64)
     a_tok = np.asarray(a_tok, dtype=np.int64)
@@ -416,7 +419,12 @@ def combine(tokens, a_tok, a_exp, a_w, expert_out, residual=None,
             term = float(a_w[a]) * expert_out(a)
             acc = term if acc is None else acc + term
         rows.append(acc)
-    return np.stack(rows)
+    if d is None:
+        widths = [r.shape[0] for r in rows if r is not None]
+        if not widths:
+            raise ValueError("no token has a term: pass the model width d")
+        d = widths[0]
+    return np.stack([np.zeros(d) if r is None else r for r in rows])
 
 
 # --------------------------------------------------------------------------
@@ -519,7 +527,7 @@ def forward(cfg, x, W1, W2, sel, kinds=None, const_vecs=None, Ws1=None,
     if Ws1 is not None:
         shared = mlp_gelu(_f64(x[tokens]), Ws1, Ws2)
     return combine(tokens, a_tok, a_exp, a_w, lambda a: out[int(a)],
-                   residual=residual, shared_out=shared)
+                   residual=residual, shared_out=shared, d=x.shape[1])
 
 
 def dense_masked_forward(cfg, x, W1, W2, A, mask, kinds=None,

@@ -315,6 +315,29 @@ def test_empty_slots_contribute_nothing():
     assert offsets.tolist() == [0, 1, 2, 3] and row_of.tolist() == [1, -1, 0, 2]
 
 
+def test_unpicked_token_sums_to_zero():
+    # Expert choice can leave a token unpicked. Its output is the empty sum
+    # over its experts: 0 without a residual, the residual row with one;
+    # picked tokens keep their weighted expert sums.
+    cfg = {"routing": "expert_choice", "E": 2, "h": 3, "act": "gelu"}
+    rng = np.random.default_rng(25)
+    x = rng.normal(size=(4, 5))
+    W1 = rng.normal(size=(2, 3, 5))
+    W2 = rng.normal(size=(2, 5, 3))
+    # one group of 4 tokens, C = 1: expert 0 takes token 2, expert 1 token 0
+    sel = {"tok": np.array([[[2], [0]]]), "w": np.array([[[0.25], [0.5]]])}
+    y = om.forward(cfg, x, W1, W2, sel)
+    assert y.shape == (4, 5)
+    np.testing.assert_array_equal(y[[1, 3]], np.zeros((2, 5)))
+    np.testing.assert_allclose(y[2], 0.25 * om.mlp_gelu(x[2:3], W1[0], W2[0])[0], rtol=1e-12)
+    np.testing.assert_allclose(y[0], 0.5 * om.mlp_gelu(x[0:1], W1[1], W2[1])[0], rtol=1e-12)
+    yr = om.forward(cfg, x, W1, W2, sel, residual=x)
+    np.testing.assert_array_equal(yr[[1, 3]], x[[1, 3]])
+    np.testing.assert_allclose(yr[[0, 2]], x[[0, 2]] + y[[0, 2]], rtol=1e-12)
+    # a subset made only of unpicked tokens still has the model width
+    assert om.forward(cfg, x, W1, W2, sel, tokens=[3, 1]).tolist() == [[0.0] * 5] * 2
+
+
 # ---------------------------------------------------------------- dispatch
 def test_dispatch_hand_example():
     # Token choice, T=3, k=2, experts 0..2 heavy, 3 is zero-compute.
