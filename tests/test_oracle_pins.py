@@ -404,6 +404,25 @@ def test_mlp_rank_one_closed_form():
     np.testing.assert_allclose(y2, expect2, rtol=1e-13)
 
 
+def test_swiglu_expert_takes_gate_rows_first():
+    # A SwiGLU expert's W1 block holds its h gate rows, then its h up rows:
+    # with h = 2, y = W2 (silu(Wg x) * (Wu x)) written out by hand. Swapping
+    # the halves gives silu(Wu x) * (Wg x), which differs.
+    rng = np.random.default_rng(26)
+    d, h = 5, 2
+    W1e = rng.normal(size=(2 * h, d))
+    W2e = rng.normal(size=(d, h))
+    X = rng.normal(size=(3, d))
+    y = om.heavy_expert("swiglu", X, W1e, W2e, h)
+    for i in range(3):
+        gate = W1e[:h] @ X[i]
+        up = W1e[h:] @ X[i]
+        hid = gate * expit(gate) * up
+        np.testing.assert_allclose(y[i], W2e @ hid, rtol=1e-13)
+        swapped = up * expit(up) * gate
+        assert not np.allclose(y[i], W2e @ swapped)
+
+
 def test_mlp_identity_weights_give_activation():
     X = np.linspace(-3, 3, 12).reshape(3, 4)
     np.testing.assert_allclose(om.mlp_gelu(X, np.eye(4), np.eye(4)), X * ndtr(X), rtol=1e-14)
