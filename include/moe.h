@@ -310,7 +310,10 @@ MOE_API int moe_grouped_mlp(const moe_config *cfg, const void *x_perm,
  * With cfg->const_mix a constant expert's term is a0 x_s + a1 v_c,
  * (a0, a1) = softmax(Wc_c x_s); its x part is added after the slots.
  * `residual` may be the same buffer as `y` (the sum is formed element by
- * element before y is written).
+ * element before y is written). A token with no assignment (expert choice
+ * may leave a token unpicked) gets r_s + y_shared[s], 0 without either; an
+ * assignment whose row_of is -1 or whose expert id is out of range adds
+ * nothing.
  *   sel, w       the selection (as in moe_dispatch) and its [n_assign] weights
  *   row_of       from moe_dispatch;  tok_ptr/tok_assign: expert choice only
  *   x            [T, d] (identity experts); const_vecs [n_const, d]
