@@ -181,3 +181,23 @@ def test_exchange_plan_splits_and_received_experts():
     assert p1.recv_expert.tolist() == [0, 0, 0, 1] + [1, 1]
     # what one rank sends to another is what that rank receives from it
     assert p0.send[1] == p1.recv[0] and p1.send[0] == p0.recv[1]
+
+
+def test_shard_bounds_partition_the_experts():
+    for n in range(0, 20):
+        for world in range(1, 9):
+            shard = ExpertShard(n, world)
+            b = [shard.bounds(r) for r in range(world)]
+            assert b[0][0] == 0 and b[-1][1] == n
+            assert all(b[r][1] == b[r + 1][0] for r in range(world - 1))
+            sizes = [hi - lo for lo, hi in b]
+            assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)
+
+
+def test_cuda_steps_take_token_choice_only():
+    # Expert-choice groups and DES blocks shard as replicas, not by expert.
+    from mixture_experts_layer_33_b200.expert_parallel import CudaOps
+    from mixture_experts_layer_33_b200 import inputs as gen
+    for name in ("ecdit", "des_vote"):
+        with pytest.raises(ValueError):
+            CudaOps(gen.workload(name), ExpertShard(4, 2), 0, None, None, None, device="cpu")
