@@ -365,25 +365,19 @@ class StagedLayer:
         mark(4)
 
 
-def gpu_bench(args):
+# The other workloads measured beside the headline one, each timed exactly
+# like it (the CPU oracle is timed for the headline workload only).
+SECONDARY_WORKLOADS = ("ecdit", "des_vote", "mmoe", "mmoe_skewed", "tiny_fp32")
+
+
+def measure_workload(m, gen, name, dev, args, world, dist, rank):
+    """One workload: the layer as a CUDA graph (value), the staged calls
+    (stage split and the dominant kernel's roofline), the fused one-launch
+    layers eagerly, and the host-buffer path (e2e). Returns the fields of
+    its JSON line and the host inputs (for the CPU oracle)."""
     import torch
-    import torch.distributed as dist
 
-    from mixture_experts_layer_33_b200 import inputs as gen
-    from mixture_experts_layer_33_b200 import moe as m
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    if m.device_check(local) != m.MOE_OK:
-        raise RuntimeError("not an sm_100 GPU")
-
-    cfg = gen.workload(args.workload)
+    cfg = gen.workload(name)
     inp = gen.make_inputs(cfg, dev)
     layer = StagedLayer(m, cfg, inp, dev)
     flush = L2Flush(dev)
@@ -394,7 +388,7 @@ def gpu_bench(args):
         layer.run()
     torch.cuda.synchronize()
     if int(layer.status.item()) != 0:
-        raise RuntimeError(f"device status {int(layer.status.item())}")
+        raise RuntimeError(f"device status {int(layer.status.item())} ({name})")
 
     # Executed heavy rows and used experts (fixed by the seeded inputs).
     offs = layer.offsets.cpu().tolist()
@@ -444,6 +438,8 @@ def gpu_bench(args):
     max_s = reduce_max_over_ranks(total_ms / 1e3, dist if world > 1 else None)
     ms_per_step = max_s * 1e3 / args.steps
     value = aggregate_throughput(cfg["T"] * args.steps, world, max_s)
+    graphed = graph is not None
+    del graph
 
     # Timed region 2: the same passes as staged calls with an event between
     # stages, for the per-stage split and the dominant kernel's duration.
@@ -500,6 +496,8 @@ def gpu_bench(args):
     e2e_s = reduce_max_over_ranks(e2e_ms / 1e3, dist if world > 1 else None)
     act_bytes = cfg["T"] * cfg["d"] * inp["x"].element_size()
     h2d = act_bytes + (cfg["T"] * cfg["E"] * 4 if zp_h is not None else 0)
+    if int(layer.status.item()) != 0:
+        raise RuntimeError(f"device status {int(layer.status.item())} ({name})")
 
     peaks, peak_src = load_peaks()
     tr = NCU_TRAFFIC.get(cfg["name"])
@@ -509,7 +507,7 @@ def gpu_bench(args):
         # One kernel on CUDA cores: fp32 FMAs against the fp32 lanes' peak at
         # the maximum SM clock (latency-bound at these sizes).
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        pk = sms * FP32_LANES_PER_SM * 2 * clocks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        pk = sms * FP32_LANES_PER_SM * 2 * (clocks.get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
         achieved = flops / (fused_ms / 1e3) / 1e12
         roof = {"bound": "alu", "kernel": "small_f32_kernel (whole layer, one launch after a memset)",
                 "achieved": round(achieved, 2), "peak": round(pk, 1), "unit": "TFLOP/s",
@@ -521,9 +519,7 @@ def gpu_bench(args):
             kname = "moe_block_kernel (whole layer, one launch after a memset)"
             achieved = bytes_ / (fused_ms / 1e3) / 1e9
         else:
-            kname = ("expert_stream_kernel (weight-streaming expert MLP, one launch)"
-                     if cfg["T"] <= 128 and cfg["dtype"] == "bf16"
-                     else "grouped_mlp (GEMM1 + GEMM2 launches)")
+            kname = "expert_stream_kernel (weight-streaming expert MLP, one launch)"
             achieved = bytes_ / (gm_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "kernel": kname,
                 "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -537,17 +533,12 @@ def gpu_bench(args):
                 "frac": round(achieved / pk, 4), "traffic": traffic,
                 "algorithmic_per_launch": flops, "peak_source": peak_src + " (burst)"}
 
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": cfg["dtype"], "data": "synthetic (seeded Gaussian inputs, random-init weights)",
-        "config": {"workload": describe(cfg), "global_batch_tokens": cfg["T"] * world,
-                   "parallelism": "replicas" if world > 1 else "single GPU",
-                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so L2 is left clean)"},
+    out = {
+        "value": round(value, 1), "unit": "tokens/s", "ms_per_step": round(ms_per_step, 4),
+        "dtype": cfg["dtype"], "config": bench_config(cfg, world),
         "layer_tflops": round(flops / (ms_per_step / 1e3) / 1e12, 1),
         "layer_weight_gbs": round(weight_bytes_used(cfg, used) / (ms_per_step / 1e3) / 1e9, 1),
-        "cuda_graph": graph is not None,
+        "cuda_graph": graphed,
         "stage_ms": {k: round(v / args.steps, 4) for k, v in stage_ms.items()},
         "fused_layer_ms": round(fused_ms, 4) if fused_ms is not None else None,
         "heavy_rows": n_rows, "experts_used": used,
@@ -558,9 +549,53 @@ def gpu_bench(args):
         "gpu_launches": forward_launches(cfg) * args.steps,
         "clocks": clocks,
     }
+    hin = {k: gen.to_numpy_f32(v) for k, v in inp.items()} if rank == 0 else None
+    del layer, inp, ws, flush
+    torch.cuda.empty_cache()
+    return cfg, out, hin
+
+
+def bench_config(cfg, world):
+    """The ``config`` object of a JSON line (the same for both arms)."""
+    return {"workload": describe(cfg), "global_batch_tokens": cfg["T"] * world,
+            "parallelism": "replicas" if world > 1 else "single GPU",
+            "l2": "flushed before every timed step (256 MiB write, then 256 MiB read so L2 is left clean)"}
+
+
+def gpu_bench(args):
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_33_b200 import inputs as gen
+    from mixture_experts_layer_33_b200 import moe as m
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if m.device_check(local) != m.MOE_OK:
+        raise RuntimeError("not an sm_100 GPU")
+
+    cfg, res, hin = measure_workload(m, gen, args.workload, dev, args, world, dist, rank)
+    line = {"metric": METRIC, "value": res["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": res["dtype"], "data": "synthetic (seeded Gaussian inputs, random-init weights)"}
+    line.update({k: v for k, v in res.items() if k not in line})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, {k: gen.to_numpy_f32(v) for k, v in inp.items()},
-                                            budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(cfg, hin, budget_s=args.cpu_budget)
+    hin = None
+    if args.workload == DEFAULT_WORKLOAD and not args.headline_only:
+        # The other workloads, each timed like the headline one; the total
+        # launches of the run include theirs.
+        line["workloads"] = {}
+        for name in SECONDARY_WORKLOADS:
+            _, r2, _ = measure_workload(m, gen, name, dev, args, world, dist, rank=1)
+            line["workloads"][name] = r2
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -647,10 +682,15 @@ def reference_bench(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": describe(cfg)},
+        "config": bench_config(cfg, world),
         "cpu_baseline": {"value": round(v, 2), "unit": "tokens/s", "cores": _cores(),
                          "kind": "oracle",
-                         "sample": f"first {done} of {cfg['T']} tokens per step"},
+                         "sample": (f"fp64 numpy oracle, own routing, first {done} of {cfg['T']} "
+                                    "tokens per step (a token's output depends only on its own "
+                                    "routing under token choice, so any prefix is exact)"
+                                    if cfg["routing"] == "token_topk" else
+                                    f"fp64 numpy oracle, own routing, first {done} of {cfg['T']} "
+                                    "tokens per step (whole routing groups / blocks)")},
         "e2e": {"value": round(v, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "torch_threads": torch.get_num_threads(),
@@ -802,6 +842,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches, not a CUDA graph")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="measure the named workload only (no 'workloads' entries)")
     ap.add_argument("--des-sweep", action="store_true",
                     help="vanilla vs DES-Seq vs DES-Vote over block sizes (one JSON line)")
     ap.add_argument("--ec-sweep", action="store_true",

@@ -25,11 +25,18 @@
  *     are OR-ed into the caller's int32 status word `dev_status` (device
  *     memory, nullable) as MOE_DEV_* bits; the offending item is skipped,
  *     nothing traps.
- *   - The library allocates no memory. Scratch comes from a caller
- *     workspace of at least moe_workspace_size() bytes, 256-byte aligned.
- *     Calls that share a workspace must not overlap on the device.
- *   - There is no global mutable state: calls on different streams with
- *     different workspaces may run concurrently.
+ *   - The library allocates no memory on a call's path. Scratch comes from
+ *     a caller workspace of at least moe_workspace_size() bytes, 256-byte
+ *     aligned. Calls that share a workspace must not overlap on the device.
+ *     Two exceptions, each documented at its entry point: the
+ *     allocation-free dispatch (moe_dispatch_noalloc) keeps its scratch in
+ *     one fixed library-owned device array per GPU, shared by all its
+ *     calls; and moe_forward_host creates two library-owned side streams
+ *     and events per device on its first pipelined call and keeps them for
+ *     the life of the process.
+ *   - Apart from those two and from one-time lookups made safely on first
+ *     use, there is no global mutable state: calls on different streams
+ *     with different workspaces may run concurrently.
  *
  * Expert ids: heavy (MLP) experts occupy ids [0, n_heavy); ids
  * [n_heavy, E) are zero-computation experts whose kinds are listed in
@@ -260,12 +267,15 @@ MOE_API int moe_dispatch(const moe_config *cfg, const int32_t *sel, const void *
  *   - It allocates nothing. Its scratch (the per-block expert histograms)
  *     is a fixed file-scope __device__ array of MOE_NOALLOC_SCRATCH_BYTES
  *     that every GPU loading the library holds until the process exits.
- *   - Limit: ceil(n_assign / 1024) * n_heavy * 4 bytes must fit in
- *     MOE_NOALLOC_SCRATCH_BYTES; larger configurations return
+ *   - Limit: max(1, ceil(n_assign / 1024)) * max(1, n_heavy) * 4 bytes
+ *     must fit in MOE_NOALLOC_SCRATCH_BYTES; larger configurations return
  *     MOE_ERR_UNSUPPORTED before anything is launched (use moe_dispatch).
  *   - The first call on a device, made with that device current, looks up
  *     the array's device address once (cudaGetSymbolAddress) and caches
- *     it; make that first call before any stream capture.
+ *     it for that device's current CUDA context; make that first call
+ *     before any stream capture. A device reset ends the context: the
+ *     first call after it (in the new context) looks the address up again,
+ *     so it too belongs before any capture.
  *   - All calls share the one array and it keeps the last call's contents
  *     (the kernels overwrite every entry they read, so nothing needs
  *     clearing). Calls that overlap on the GPU race on it: serialise them.
@@ -341,6 +351,25 @@ MOE_API int moe_combine(const moe_config *cfg, const void *y_perm,
  */
 MOE_API int moe_activation(const float *x, float *y, int64_t n, int act,
                            moe_stream_t stream);
+
+/*
+ * Test hook for failure detection (no counterpart on the pages). Blocks of
+ * at most 128 bf16 tokens with a shared expert finish their routing in one
+ * cooperative kernel whose CTAs meet at grid barriers (software barriers
+ * on a global counter, each wait bounded by 2 s). This sets, for every
+ * later launch of that kernel in the process, the wait limit to `limit_ns`
+ * (0 restores the 2 s default) and makes the barriers wait for
+ * `extra_arrivals` arrivals beyond the grid (0 restores the default), so a
+ * test can make a wait expire on purpose without faulting or hanging the
+ * GPU. An expired barrier sets MOE_DEV_TIMEOUT in dev_status, and the
+ * CTAs that gave up leave their tokens' slots empty (expert -1, weight 0,
+ * no row) and zero row offsets (CTA 0), so the rest of the layer runs on
+ * an empty routing for those tokens: y = residual + shared expert there.
+ * Process-wide; set it only while no layer call is being enqueued.
+ *   limit_ns        0 .. 2e9;  extra_arrivals  0 .. 1024
+ * Returns MOE_ERR_INVALID_ARG outside those ranges.
+ */
+MOE_API int moe_test_set_barrier_wait(uint64_t limit_ns, int extra_arrivals);
 
 /* Optional outputs of moe_forward (each pointer nullable; device memory). */
 typedef struct moe_forward_aux {

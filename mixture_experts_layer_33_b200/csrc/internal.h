@@ -78,9 +78,15 @@ struct SmallRouteArgs {
   unsigned *barrier;     // grid-barrier counter, zeroed before the launch
   unsigned *gmask;       // [n_heavy][4] token bitmasks, zeroed before the launch
   int32_t *dev_status;
+  // Set by launch_small_route: the grid barriers' wait limit and the
+  // arrivals they wait for beyond the grid (0 except under the test hook).
+  unsigned long long wait_ns;
+  int extra_arrivals;
 };
 bool small_route_supported(int T, int E, int k, int routing, int dtype);
 int launch_small_route(const SmallRouteArgs &args, cudaStream_t stream);
+// Test hook behind moe_test_set_barrier_wait (0, 0 restores the defaults).
+void set_small_route_test_wait(unsigned long long limit_ns, int extra_arrivals);
 
 // block_sm100.cu: the whole layer for blocks of <= 128 bf16 tokens (token
 // choice or DES-Vote, no shared expert) in one persistent cooperative

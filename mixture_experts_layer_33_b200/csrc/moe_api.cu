@@ -688,6 +688,13 @@ int moe_activation(const float *x, float *y, int64_t n, int act, moe_stream_t st
   return launch_activation(x, y, n, act, stream);
 }
 
+int moe_test_set_barrier_wait(uint64_t limit_ns, int extra_arrivals) {
+  if (limit_ns > 2000000000ull || extra_arrivals < 0 || extra_arrivals > 1024)
+    return MOE_ERR_INVALID_ARG;
+  set_small_route_test_wait((unsigned long long)limit_ns, extra_arrivals);
+  return MOE_OK;
+}
+
 int moe_forward(const moe_config *cfg, const void *x, const void *residual, const float *z_prev,
                 const void *W_r, const float *bias, const void *W1, const void *W2,
                 const void *Ws1, const void *Ws2, const void *const_vecs, void *y,

@@ -9,7 +9,10 @@
 //     bias and gate residual, softmax, then either the token-choice top-k
 //     or the DES-Vote top-K votes (exact int64 fixed point, atomics).
 //     Token choice also marks its picks in per-expert token bitmasks.
-//   grid barrier (bounded wait).
+//   grid barrier (bounded wait; on expiry the CTA flags MOE_DEV_TIMEOUT,
+//     leaves its token's slots empty -- expert -1, weight 0, no row -- and,
+//     in CTA 0, zero row offsets, so the later stages of the layer see an
+//     empty, in-bounds routing for what did not finish).
 //   DES only: every CTA re-runs the same election from the summed votes,
 //     re-routes its own token over the core set, marks its picks in the
 //     bitmasks; second grid barrier.
@@ -37,6 +40,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -48,6 +53,11 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kMaxE = 128;
 constexpr int kXVecs = 4;  // x-row vectors held per thread from the start (rows <= 8192 bf16)
 constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;
+
+// Test hook (moe_test_set_barrier_wait): a shorter wait limit and extra
+// arrivals the grid barriers wait for, read at each launch.
+std::atomic<unsigned long long> g_test_wait_ns{0};
+std::atomic<int> g_test_extra_arrivals{0};
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
   unsigned v;
@@ -63,9 +73,10 @@ __device__ __forceinline__ uint4 ld_nc_v4(const uint4 *p) {
   return v;
 }
 
-// Grid barrier among the co-resident CTAs: arrive, then wait (bounded)
-// until `target` arrivals. Returns false if the wait expired.
-__device__ __forceinline__ bool grid_barrier(unsigned *ctr, unsigned target, int *ok_slot) {
+// Grid barrier among the co-resident CTAs: arrive, then wait (at most
+// `limit_ns`) until `target` arrivals. Returns false if the wait expired.
+__device__ __forceinline__ bool grid_barrier(unsigned *ctr, unsigned target, uint64_t limit_ns,
+                                             int *ok_slot) {
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -74,7 +85,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned *ctr, unsigned target, int
     if (ld_acquire_u32(ctr) < target) {
       const uint64_t t0 = global_timer_ns();
       while (ld_acquire_u32(ctr) < target) {
-        if (global_timer_ns() - t0 > kBarrierTimeoutNs) { ok = 0; break; }
+        if (global_timer_ns() - t0 > limit_ns) { ok = 0; break; }
         __nanosleep(32);
       }
     }
@@ -82,6 +93,22 @@ __device__ __forceinline__ bool grid_barrier(unsigned *ctr, unsigned target, int
   }
   __syncthreads();
   return *ok_slot != 0;
+}
+
+// After an expired barrier: flag the timeout and leave this CTA's token
+// with empty slots (and, in CTA 0, zero row offsets) so that the dispatch
+// outputs the later stages read stay in bounds. CTA-wide.
+__device__ __forceinline__ void abandon_token(const SmallRouteArgs &a, int t) {
+  const int tid = threadIdx.x;
+  if (tid == 0) set_status(a.dev_status, MOE_DEV_TIMEOUT);
+  if (tid < a.k) {
+    const int i = t * a.k + tid;
+    a.sel[i] = -1;
+    a.w[i] = 0.f;
+    a.row_of[i] = -1;
+  }
+  if (t == 0)
+    for (int e = tid; e <= a.n_heavy; e += kThreads) a.offsets[e] = 0;
 }
 
 // DES election, identical in every CTA: the M_core largest vote totals
@@ -246,8 +273,8 @@ small_route_kernel(SmallRouteArgs a) {
     }
   }
 
-  if (!grid_barrier(a.barrier, T, &barrier_ok)) {
-    if (tid == 0) set_status(a.dev_status, MOE_DEV_TIMEOUT);
+  if (!grid_barrier(a.barrier, T + a.extra_arrivals, a.wait_ns, &barrier_ok)) {
+    abandon_token(a, t);
     return;
   }
 
@@ -269,8 +296,8 @@ small_route_kernel(SmallRouteArgs a) {
         if (e < a.n_heavy) atomicOr(a.gmask + 4 * e + (t >> 5), 1u << (t & 31));
       }
     }
-    if (!grid_barrier(a.barrier, 2 * T, &barrier_ok)) {
-      if (tid == 0) set_status(a.dev_status, MOE_DEV_TIMEOUT);
+    if (!grid_barrier(a.barrier, 2 * T + 2 * a.extra_arrivals, a.wait_ns, &barrier_ok)) {
+      abandon_token(a, t);
       return;
     }
   } else {
@@ -342,9 +369,18 @@ bool small_route_supported(int T, int E, int k, int routing, int dtype) {
          k <= kSmallRouteMaxK && (int64_t)T * k <= kSmallRouteMaxAssign;
 }
 
-int launch_small_route(const SmallRouteArgs &a, cudaStream_t stream) {
-  if (a.T == 0) return MOE_OK;
-  if (!small_route_supported(a.T, a.E, a.k, a.routing, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
+void set_small_route_test_wait(unsigned long long limit_ns, int extra_arrivals) {
+  g_test_wait_ns.store(limit_ns);
+  g_test_extra_arrivals.store(extra_arrivals);
+}
+
+int launch_small_route(const SmallRouteArgs &args, cudaStream_t stream) {
+  if (args.T == 0) return MOE_OK;
+  if (!small_route_supported(args.T, args.E, args.k, args.routing, MOE_BF16)) return MOE_ERR_UNSUPPORTED;
+  SmallRouteArgs a = args;
+  const unsigned long long test_ns = g_test_wait_ns.load();
+  a.wait_ns = test_ns ? test_ns : kBarrierTimeoutNs;
+  a.extra_arrivals = g_test_extra_arrivals.load();
   cudaLaunchConfig_t cfg;
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(a.T);

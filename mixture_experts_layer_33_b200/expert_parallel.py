@@ -27,11 +27,24 @@ experts [lo_p, hi_p)):
    applies unchanged (shared expert, residual and zero-computation experts
    are local to the token's rank).
 
+`InterweavedEP` is DICE's interweaved schedule over the same steps (Key
+designs, "Interweaved Parallelism"): the dispatch exchange completes within
+the step (fresh), while the combine exchange of a step's expert outputs is
+started asynchronously and consumed one step later, so the routed-expert
+part of a step's output comes from the previous step (one step stale) and
+only those combine results are cached. The reading taken where the page is
+brief: the stale part is the sum over the previous step's heavy-expert
+slots of weight times expert output, with that step's routing; everything
+local to the token's rank (residual, shared expert, zero-computation
+experts) uses the current step's input and routing; the first step, with
+nothing cached, runs synchronously.
+
 Every compute step is an `Ops` call: `CudaOps` runs the library's kernels
 through the C ABI (one GPU per rank, NCCL); the tests drive the same
-orchestration with the fp64 oracle on CPU ranks over gloo. The collectives
-are plain `torch.distributed` calls; the fused dispatch/combine kernels over
-NVLink peer memory are not built.
+orchestration with the fp64 oracle on CPU ranks over gloo, and `CudaOps` on
+one GPU as a one-rank NCCL group. The collectives are plain
+`torch.distributed` calls; the fused dispatch/combine kernels over NVLink
+peer memory are not built.
 """
 
 from __future__ import annotations
@@ -85,10 +98,10 @@ def _all_gather_counts(counts: np.ndarray, device, group) -> np.ndarray:
     return torch.stack(out).cpu().numpy()
 
 
-def ep_forward(ops, shard: ExpertShard, x, residual=None, z_prev=None, group=None):
-    """The layer on this rank's tokens `x` (and their previous-layer logits
-    `z_prev` under MMOE's gate residual) with the heavy experts sharded over
-    `group`; returns this rank's outputs."""
+def _route_dispatch_compute(ops, shard: ExpertShard, x, z_prev, group):
+    """Steps 1-3: route, dispatch, the dispatch exchange (completed here)
+    and this rank's experts on the rows it received. Returns the routing,
+    the send/receive splits and the expert outputs in received order."""
     rank = dist.get_rank(group)
     sel, w = ops.route(x, z_prev)
     x_perm, offsets, row_of = ops.dispatch(sel, x)
@@ -104,9 +117,83 @@ def ep_forward(ops, shard: ExpertShard, x, residual=None, z_prev=None, group=Non
         x_grp, offs_grp, row_of_grp, sel_recv = ops.regroup(x_recv, plan.recv_expert)
         y_grp = ops.experts(x_grp, offs_grp)
         y_recv = ops.ungroup(y_grp, row_of_grp, sel_recv, x_recv)
-    y_back = ops.empty(n_send, d)
+    return sel, w, row_of, plan, n_send, y_recv
+
+
+def ep_forward(ops, shard: ExpertShard, x, residual=None, z_prev=None, group=None):
+    """The layer on this rank's tokens `x` (and their previous-layer logits
+    `z_prev` under MMOE's gate residual) with the heavy experts sharded over
+    `group`; returns this rank's outputs. Raises if a device step flagged
+    an error (bad ids, an expired bounded wait)."""
+    sel, w, row_of, plan, n_send, y_recv = _route_dispatch_compute(ops, shard, x, z_prev, group)
+    y_back = ops.empty(n_send, x.shape[1])
     dist.all_to_all_single(y_back, y_recv.contiguous(), plan.send, plan.recv, group=group)
-    return ops.combine(y_back, ops.shared(x), sel, w, row_of, x, residual)
+    y = ops.combine(y_back, ops.shared(x), sel, w, row_of, x, residual)
+    ops.check_status()
+    return y
+
+
+def merge_stale_slots(prev_sel, prev_w, prev_row_of, sel, w, n_heavy, k):
+    """Slot lists of the interweaved combine, 2k slots per token: first the
+    previous step's k slots with only their heavy experts kept (their rows
+    index the previous step's returned expert outputs), then this step's k
+    slots with only the zero-computation experts kept. A dropped slot is
+    expert -1 with no row, which the combine skips. Index and weight
+    bookkeeping only: the sums are the combine's."""
+    prev_sel, sel = prev_sel.reshape(-1, k), sel.reshape(-1, k)
+    heavy_prev = (prev_sel >= 0) & (prev_sel < n_heavy)
+    light_now = sel >= n_heavy
+    minus1 = torch.full_like(sel, -1)
+    m_sel = torch.cat([torch.where(heavy_prev, prev_sel, minus1),
+                       torch.where(light_now, sel, minus1)], dim=1)
+    m_w = torch.cat([prev_w.reshape(-1, k), w.reshape(-1, k)], dim=1)
+    prev_row = torch.as_tensor(np.asarray(prev_row_of)) if not isinstance(prev_row_of, torch.Tensor) \
+        else prev_row_of
+    prev_row = prev_row.to(sel.device).reshape(-1, k)
+    m_row = torch.cat([torch.where(heavy_prev, prev_row.to(sel.dtype), minus1), minus1], dim=1)
+    return m_sel.reshape(-1).contiguous(), m_w.reshape(-1).contiguous(), m_row.reshape(-1).contiguous()
+
+
+class InterweavedEP:
+    """DICE's interweaved expert-parallel schedule: fresh dispatch, combine
+    one step stale (see the module docstring). Call `step` once per
+    diffusion step for this layer, then `finish` before the process group
+    goes away; every rank takes the same collective steps in the same
+    order (one counts all-gather, one dispatch exchange and one combine
+    exchange, started asynchronously, per step)."""
+
+    def __init__(self, ops, shard: ExpertShard, group=None):
+        self.ops, self.shard, self.group = ops, shard, group
+        self.pending = None  # the previous step's combine exchange and routing
+
+    def step(self, x, residual=None, z_prev=None):
+        ops = self.ops
+        sel, w, row_of, plan, n_send, y_recv = _route_dispatch_compute(
+            ops, self.shard, x, z_prev, self.group)
+        y_back = ops.empty(n_send, x.shape[1])
+        y_recv = y_recv.contiguous()
+        work = dist.all_to_all_single(y_back, y_recv, plan.send, plan.recv, group=self.group,
+                                      async_op=True)
+        prev, self.pending = self.pending, (work, y_back, y_recv, sel, w, row_of)
+        y_sh = ops.shared(x)
+        if prev is None:
+            # nothing cached yet: this step's own combine, synchronously
+            work.wait()
+            y = ops.combine(y_back, y_sh, sel, w, row_of, x, residual)
+        else:
+            p_work, p_back, _, p_sel, p_w, p_row = prev
+            p_work.wait()
+            k = int(sel.numel()) // max(1, x.shape[0])
+            m_sel, m_w, m_row = merge_stale_slots(p_sel, p_w, p_row, sel, w, ops.n_heavy, k)
+            y = ops.combine(p_back, y_sh, m_sel, m_w, m_row, x, residual, k=2 * k)
+        ops.check_status()
+        return y
+
+    def finish(self):
+        """Wait for the last step's combine exchange (its result is unused)."""
+        if self.pending is not None:
+            self.pending[0].wait()
+            self.pending = None
 
 
 class CudaOps:
@@ -114,9 +201,9 @@ class CudaOps:
 
     `cfg` is the layer's configuration (token choice) over all experts;
     `W1_local` / `W2_local` hold this rank's experts only (heavy experts
-    [lo, hi) of `shard`), in the same layouts as the full tensors. Not run
-    on a GPU here (one GPU per run); the orchestration is covered on CPU
-    ranks with the oracle's steps.
+    [lo, hi) of `shard`), in the same layouts as the full tensors. Run on
+    one GPU as a one-rank NCCL group (the exchanges are then copies to
+    itself); more ranks are covered on CPU ranks with the oracle's steps.
     """
 
     def __init__(self, cfg, shard: ExpertShard, rank: int, W_r, W1_local, W2_local,
@@ -130,6 +217,7 @@ class CudaOps:
         self.W1, self.W2 = W1_local, W2_local
         lo, hi = shard.bounds(rank)
         self.n_local = hi - lo
+        self.n_heavy = shard.n_heavy
         self.dtype = torch.bfloat16 if cfg["dtype"] == "bf16" else torch.float32
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
@@ -212,9 +300,15 @@ class CudaOps:
                            self.status, ws)
         return y_sh
 
-    def combine(self, y_back, y_sh, sel, w, row_of, x, residual):
-        c = self._local_cfg(x.shape[0])
+    def combine(self, y_back, y_sh, sel, w, row_of, x, residual, k=None):
+        c = self.m.make_config(dict(self.cfg, T=x.shape[0], k=k or self.cfg["k"]))
         y = torch.empty_like(x)
         self.m.combine(c, y_back, y_sh, sel, w, row_of, None, None, x, self.cv, residual, y,
                        self.status)
         return y
+
+    def check_status(self):
+        """Raise if any step flagged an error in the device status word."""
+        st = int(self.status.item())
+        if st != 0:
+            raise RuntimeError(f"expert-parallel layer: device status {st:#x}")

@@ -30,7 +30,7 @@ ENTRY_POINTS = (
     "moe_workspace_size", "moe_router", "moe_select_topk",
     "moe_select_expert_choice", "moe_core_set_vote", "moe_core_set_union", "moe_dispatch",
     "moe_grouped_mlp", "moe_combine", "moe_forward", "moe_forward_host",
-    "moe_dispatch_noalloc", "moe_activation",
+    "moe_dispatch_noalloc", "moe_activation", "moe_test_set_barrier_wait",
 )
 NOALLOC_SCRATCH_BYTES = 256 * 1024  # MOE_NOALLOC_SCRATCH_BYTES
 
@@ -69,6 +69,7 @@ _SIGS = {
     "moe_dispatch": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_dispatch_noalloc": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_activation": (_i32, [_vp, _vp, ctypes.c_int64, _i32, _vp]),
+    "moe_test_set_barrier_wait": (_i32, [ctypes.c_uint64, _i32]),
     "moe_grouped_mlp": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                _vp]),
     "moe_combine": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -246,6 +247,14 @@ def activation(x, y, act=GELU_ERF, stream=None):
     """y = GELU(x) (act=GELU_ERF) or SiLU(x) (act=SWIGLU), fp32 device tensors."""
     _check(LIB.moe_activation(_dev_ptr(x), _dev_ptr(y), x.numel(), int(act), _stream(stream)),
            "moe_activation")
+
+
+def set_barrier_wait_for_tests(limit_ns=0, extra_arrivals=0):
+    """Test hook: the small-block routing kernel's grid-barrier wait limit
+    (ns; 0 = the 2 s default) and extra arrivals it waits for (0 = none).
+    Process-wide; see moe_test_set_barrier_wait in include/moe.h."""
+    _check(LIB.moe_test_set_barrier_wait(int(limit_ns), int(extra_arrivals)),
+           "moe_test_set_barrier_wait")
 
 
 def grouped_mlp(c: MoeConfig, x_perm, offsets, W1, W2, x, Ws1, Ws2, y_perm, y_shared,

@@ -122,3 +122,12 @@ def test_entry_points_reject_bad_sizes(m):
     assert m.LIB.moe_select_expert_choice(fake, 128, 8, 64, 65, fake, fake, None) == 1
     assert m.LIB.moe_core_set_vote(fake, 32, 64, 8, 4, fake, fake, fake, fake, None) == 1
     assert m.LIB.moe_core_set_vote(fake, 32, 300, 8, 32, fake, fake, fake, fake, None) == 2
+
+
+def test_barrier_wait_hook_checks_its_arguments(m):
+    # host-side checks only; valid values just set the hook (no launch)
+    assert m.LIB.moe_test_set_barrier_wait(2_000_000_001, 0) == 1  # MOE_ERR_INVALID_ARG
+    assert m.LIB.moe_test_set_barrier_wait(0, -1) == 1
+    assert m.LIB.moe_test_set_barrier_wait(0, 1025) == 1
+    assert m.LIB.moe_test_set_barrier_wait(1000, 1) == 0
+    assert m.LIB.moe_test_set_barrier_wait(0, 0) == 0

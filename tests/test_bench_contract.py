@@ -26,6 +26,9 @@ def _check_line(d, n_gpus):
     assert d["ms_per_step"] > 0 and d["scaling"] == "weak" and d["vs_baseline"] is None
     assert d["dtype"] == "f64" and d["data"] == "synthetic"
     assert d["config"]["workload"].startswith("tiny_fp32")
+    # the same config object as the CUDA arm's line
+    assert set(d["config"]) == {"workload", "global_batch_tokens", "parallelism", "l2"}
+    assert d["config"]["global_batch_tokens"] == 256 * n_gpus
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     e = d["e2e"]

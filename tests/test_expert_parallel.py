@@ -16,7 +16,8 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from mixture_experts_layer_33_b200.expert_parallel import ExpertShard, ep_forward, exchange_plan
+from mixture_experts_layer_33_b200.expert_parallel import (ExpertShard, InterweavedEP, ep_forward,
+                                                           exchange_plan)
 from oracle import moe_oracle as om
 
 H, I, Z, C = om.HEAVY, om.IDENTITY, om.ZERO, om.CONST
@@ -36,6 +37,7 @@ class OracleOps:
     def __init__(self, cfg, shard, rank, W, kinds):
         self.cfg, self.kinds, self.W = cfg, kinds, W
         self.n_heavy = sum(1 for k in kinds if k == H)
+        assert self.n_heavy == shard.n_heavy
         lo, hi = shard.bounds(rank)
         self.n_local = hi - lo
         self.W1, self.W2 = W["W1"][lo:hi], W["W2"][lo:hi]  # the shard's experts only
@@ -75,13 +77,17 @@ class OracleOps:
             return None
         return om.mlp_gelu(x.numpy(), self.W["Ws1"], self.W["Ws2"])
 
-    def combine(self, y_back, y_sh, sel, w, row_of, x, residual):
-        T, k = x.shape[0], self.cfg["k"]
+    def check_status(self):
+        pass  # no device status on the CPU ranks
+
+    def combine(self, y_back, y_sh, sel, w, row_of, x, residual, k=None):
+        T, k = x.shape[0], k or self.cfg["k"]
         sel, xs, yb = sel.numpy(), x.numpy(), y_back.numpy()
+        row_of = np.asarray(row_of)
         cidx = np.cumsum([kd == C for kd in self.kinds]) - 1
 
         def out(a):
-            e = int(sel[a])
+            e = int(sel[a])  # never -1: the oracle's combine skips empty slots
             if self.kinds[e] == H:
                 return yb[row_of[a]]
             if self.kinds[e] == I:
@@ -165,6 +171,94 @@ def test_expert_parallel_matches_one_device_layer(case):
     y_ref = _reference(cfg, kinds, W, x, z_prev)
     for rank, lo, hi, y in got:
         np.testing.assert_allclose(y, y_ref[lo:hi], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------ interweaved (one step stale)
+N_STEPS = 3
+
+
+def _step_input(x0, t):
+    """Diffusion-step inputs: each step moves the activations a little."""
+    rng = np.random.default_rng(1000 + t)
+    return x0 + 0.3 * t * rng.normal(size=x0.shape)
+
+
+def _only(sel_idx, keep):
+    """The selection with the slots `keep` rejects emptied (expert -1)."""
+    out = dict(sel_idx)
+    out["idx"] = np.where(keep(sel_idx["idx"]), sel_idx["idx"], -1)
+    return out
+
+
+def _interweaved_reference(cfg, kinds, W, xs, zs):
+    """Step 0: the synchronous layer. Step t >= 1: residual, shared expert
+    and zero-computation experts from step t's input and routing, plus the
+    heavy experts' weighted outputs of step t-1 (its input and routing)."""
+    n_heavy = sum(1 for k in kinds if k == H)
+    outs = []
+    for t, (x, z) in enumerate(zip(xs, zs)):
+        sel = om.route(cfg, x, W["W_r"], W["bias"], z)
+        if t == 0:
+            outs.append(om.forward(cfg, x, W["W1"], W["W2"], sel, kinds, W["cv"], W["Ws1"],
+                                   W["Ws2"], residual=x))
+            continue
+        prev = om.route(cfg, xs[t - 1], W["W_r"], W["bias"], zs[t - 1])
+        stale = om.forward(cfg, xs[t - 1], W["W1"], W["W2"],
+                           _only(prev, lambda i: (i >= 0) & (i < n_heavy)), kinds, W["cv"],
+                           None, None, residual=None)
+        fresh = om.forward(cfg, x, W["W1"], W["W2"], _only(sel, lambda i: i >= n_heavy), kinds,
+                           W["cv"], W["Ws1"], W["Ws2"], residual=x)
+        outs.append(fresh + stale)
+    return outs
+
+
+def _interweaved_rank_main(rank, world, port, case, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        cfg, kinds, W, x0, z0 = _problem(case)
+        shard = ExpertShard(sum(1 for k in kinds if k == H), world)
+        lo, hi = case["T"] * rank // world, case["T"] * (rank + 1) // world
+        ep = InterweavedEP(OracleOps(cfg, shard, rank, W, kinds), shard)
+        ys = []
+        for t in range(N_STEPS):
+            x = _step_input(x0, t)
+            xt = torch.from_numpy(x[lo:hi])
+            zt = None if z0 is None else z0[lo:hi]
+            ys.append(np.asarray(ep.step(xt, residual=xt, z_prev=zt)))
+        ep.finish()
+        q.put((rank, lo, hi, ys))
+    finally:
+        dist.destroy_process_group()
+
+
+IW_CASES = [CASES[0], CASES[1], CASES[4]]
+
+
+@pytest.mark.parametrize("case", IW_CASES, ids=[c["name"] for c in IW_CASES])
+def test_interweaved_schedule_combines_one_step_stale(case):
+    world = case["world"]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_interweaved_rank_main, args=(r, world, port, case, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    cfg, kinds, W, x0, z0 = _problem(case)
+    xs = [_step_input(x0, t) for t in range(N_STEPS)]
+    zs = [z0] * N_STEPS
+    refs = _interweaved_reference(cfg, kinds, W, xs, zs)
+    for rank, lo, hi, ys in got:
+        for t in range(N_STEPS):
+            np.testing.assert_allclose(ys[t], refs[t][lo:hi], rtol=1e-12, atol=1e-12)
+        # the later steps really are stale: not the synchronous layer
+        sync = _reference(cfg, kinds, W, xs[1], z0)
+        assert not np.allclose(ys[1], sync[lo:hi], rtol=1e-6, atol=1e-6)
 
 
 def test_exchange_plan_splits_and_received_experts():

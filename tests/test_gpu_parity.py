@@ -81,8 +81,7 @@ def test_layer_small_full_oracle(name, over):
     hin = H.host(inp)
     _check_router(cfg, hin, out)
     sel = _check_selection(cfg, out)
-    y_ref = H.oracle_layer(cfg, hin, sel)
-    assert H.normwise(out["y"], y_ref) <= H.Y_TOL[cfg["dtype"]]
+    H.log_errors(f"small/{name}", *H.check_layer_outputs(cfg, inp, hin, sel, out))
 
 
 @pytest.mark.parametrize("name,over", PAIR, ids=[p[0] for p in PAIR])
@@ -94,8 +93,7 @@ def test_layer_two_sm_tiles_full_oracle(name, over):
     hin = H.host(inp)
     _check_router(cfg, hin, out)
     sel = _check_selection(cfg, out)
-    y_ref = H.oracle_layer(cfg, hin, sel)
-    assert H.normwise(out["y"], y_ref) <= H.Y_TOL[cfg["dtype"]]
+    H.log_errors(f"pair/{name}", *H.check_layer_outputs(cfg, inp, hin, sel, out))
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -111,8 +109,7 @@ def test_layer_full_size_sampled(name):
     T = cfg["T"]
     tokens = np.sort(rng.choice(T, size=min(T, 192), replace=False))
     tokens[-1] = T - 1  # include the ragged end of the last tile
-    y_ref = H.oracle_layer(cfg, hin, sel, tokens=tokens)
-    assert H.normwise(out["y"][tokens], y_ref) <= H.Y_TOL[cfg["dtype"]]
+    H.log_errors(f"full/{name}", *H.check_layer_outputs(cfg, inp, hin, sel, out, tokens=tokens))
 
 
 @pytest.mark.parametrize("name", ["ditmoe_xl", "mmoe"])
@@ -132,6 +129,87 @@ def test_independent_routing_flips_are_near_ties(name):
         kth_ref = z_ref[s, idx_ref[s, -1]]
         gpu_min = z_ref[s, idx_gpu[s]].min()
         assert abs(kth_ref - gpu_min) <= 1e-5 * scale
+
+
+def _z_ref(cfg, hin):
+    return oracle.router_logits(hin["x"], hin["W_r"], hin["logit_bias"], hin["z_prev"],
+                                cfg["gate_residual_scale"])
+
+
+def _log_affinity(z):
+    """log A = z - logsumexp(z) per token, in fp64: the ranking key of A."""
+    m = z.max(axis=1, keepdims=True)
+    return z - (m + np.log(np.exp(z - m).sum(axis=1, keepdims=True)))
+
+
+def test_independent_routing_flips_are_near_ties_expert_choice():
+    """Expert choice from the oracle's own fp64 affinities: any (group,
+    expert) whose chosen token set differs from the GPU's must differ only
+    at a near tie of the key at the C-th place (ranked on log A, so the gap
+    is measured like the logits' error)."""
+    cfg = gen.workload("ecdit")
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    hin = H.host(inp)
+    z = _z_ref(cfg, hin)
+    la = _log_affinity(z)
+    tok_ref, _ = oracle.expert_choice(np.exp(la), cfg["group_size"], cfg["capacity"])
+    S, E, C = cfg["group_size"], cfg["E"], cfg["capacity"]
+    G = cfg["T"] // S
+    tok_gpu = out["sel"].reshape(G, E, C)
+    scale = np.max(np.abs(z))
+    flips = 0
+    for g in range(G):
+        for e in range(E):
+            if np.array_equal(tok_ref[g, e], tok_gpu[g, e]):
+                continue
+            flips += 1
+            key = la[g * S:(g + 1) * S, e]
+            cth_ref = np.sort(key)[::-1][C - 1]  # the oracle's boundary key
+            gpu_min = key[tok_gpu[g, e] - g * S].min()
+            assert abs(cth_ref - gpu_min) <= 1e-5 * scale, (g, e)
+    H.log_errors(f"independent_routing/ecdit/flipped_sets={flips}", 0.0, 0.0)
+
+
+def test_independent_routing_flips_are_near_ties_des_vote():
+    """DES-Vote from the oracle's own fp64 probabilities, one decision at a
+    time, each fed the GPU's earlier decisions: (i) every token's top-K on
+    log P, (iii) the core set from the votes the oracle tallies in fp64
+    over the GPU's top-K sets, (iv) the re-route over the GPU's core set.
+    Every difference must be a near tie of its key."""
+    cfg = gen.workload("des_vote")
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    hin = H.host(inp)
+    z = _z_ref(cfg, hin)
+    la = _log_affinity(z)
+    P = np.exp(la)
+    T, M, K, Mc = cfg["T"], cfg["E"], cfg["k"], cfg["M_core"]
+    scale = np.max(np.abs(z))
+    # (i) per-token top-K, the GPU's from its own fp32 probabilities
+    P_gpu = out["probs"].astype(np.float64)
+    top_gpu = oracle.topk_token_choice(P_gpu, K)
+    top_ref = oracle.topk_token_choice(la, K)
+    for n in range(T):
+        if set(top_gpu[n]) != set(top_ref[n]):
+            assert abs(la[n, top_ref[n, -1]] - la[n, top_gpu[n]].min()) <= 1e-5 * scale, n
+    # (iii) the core set: fp64 votes over the GPU's top-K sets
+    V = np.zeros(M)
+    for n in range(T):
+        V[top_gpu[n]] += P[n, top_gpu[n]]
+    core_gpu = out["core"][:Mc]
+    order = sorted(range(M), key=lambda e: (-V[e], e))
+    core_ref = np.sort(order[:Mc])
+    if not np.array_equal(core_ref, core_gpu):
+        vth = V[order[Mc - 1]]
+        assert abs(vth - V[core_gpu].min()) <= 1e-5 * V.max()
+    # (iv) the re-route over the GPU's core set
+    idx_gpu = out["sel"].reshape(T, K)
+    for n in range(T):
+        keys = la[n, core_gpu]
+        ref = core_gpu[np.argsort(-keys, kind="stable")[:K]]
+        if set(ref) != set(idx_gpu[n]):
+            assert abs(la[n, ref[-1]] - la[n, idx_gpu[n]].min()) <= 1e-5 * scale, n
 
 
 STAGEWISE = SMALL[1:5] + [("ditmoe_xl_2sm", PAIR[0][1])]
@@ -158,10 +236,25 @@ def test_stagewise_entry_points(name, over):
              idx=sel if r == "token_topk" else None, w=w if r == "token_topk" else None)
     if r == "expert_choice":
         m.select_expert_choice(probs, cfg["group_size"], cfg["capacity"], sel, w)
+        torch.cuda.synchronize()
+        # the entry point's own outputs, against the oracle on the GPU's probabilities
+        ref_tok, ref_w = oracle.expert_choice(probs.cpu().numpy().astype(np.float64),
+                                              cfg["group_size"], cfg["capacity"])
+        np.testing.assert_array_equal(sel.cpu().numpy().reshape(ref_tok.shape), ref_tok)
+        np.testing.assert_array_equal(w.cpu().numpy().reshape(ref_w.shape).astype(np.float64),
+                                      ref_w)
     elif r == "des_vote":
         votes = torch.empty(E, dtype=torch.int64, device=dev)
         core = torch.empty(cfg["M_core"], dtype=torch.int32, device=dev)
         m.core_set_vote(probs, cfg["k"], cfg["M_core"], votes, core, sel, w)
+        torch.cuda.synchronize()
+        ref_votes, ref_core, ref_idx, ref_w = oracle.des_vote(
+            probs.cpu().numpy().astype(np.float64), cfg["k"], cfg["M_core"])
+        np.testing.assert_array_equal(votes.cpu().numpy(), ref_votes)
+        np.testing.assert_array_equal(core.cpu().numpy(), ref_core)
+        np.testing.assert_array_equal(sel.cpu().numpy().reshape(ref_idx.shape), ref_idx)
+        np.testing.assert_array_equal(w.cpu().numpy().reshape(ref_w.shape).astype(np.float64),
+                                      ref_w)
     else:
         # the standalone selection must agree with the fused one bit for bit
         sel2 = torch.empty_like(sel)
@@ -217,6 +310,82 @@ def test_stagewise_entry_points(name, over):
     assert int(status.item()) == 0
     y_ref = H.oracle_layer(cfg, hin, gsel)
     assert H.normwise(gen.to_numpy_f32(y), y_ref) <= H.Y_TOL[cfg["dtype"]]
+
+
+def _sample_rows(lo, hi, n, rng):
+    """n rows of [lo, hi): the first and last (ragged tile end) and a seeded draw."""
+    if hi - lo <= n:
+        return np.arange(lo, hi)
+    mid = rng.choice(np.arange(lo + 1, hi - 1), size=n - 2, replace=False)
+    return np.sort(np.concatenate([[lo, hi - 1], mid]))
+
+
+@pytest.mark.parametrize("name", ["ditmoe_xl", "ecdit", "mmoe"])
+def test_grouped_mlp_full_shape_sampled(name):
+    """moe_grouped_mlp alone at the full workload shape (the launch shapes
+    the layer uses: wide CTA-pair down projections at K = 4608 / 8192 / 9216,
+    the one-SM up projections), without the residual: sampled rows of four
+    experts' outputs against the oracle's expert MLP, and the shared
+    expert's output on sampled tokens."""
+    m = H.moe()
+    cfg = gen.workload(name)
+    inp = gen.make_inputs(cfg, "cuda")
+    c = m.make_config(cfg)
+    na = m.num_assignments(c)
+    T, E, d = cfg["T"], cfg["E"], cfg["d"]
+    dev = "cuda"
+    r = cfg["routing"]
+    logits = torch.empty(T, E, device=dev)
+    probs = torch.empty(T, E, device=dev)
+    sel = torch.empty(na, dtype=torch.int32, device=dev)
+    w = torch.empty(na, device=dev)
+    m.router(inp["x"], inp["W_r"], logits, probs, bias=inp["logit_bias"], z_prev=inp["z_prev"],
+             z_prev_scale=cfg["gate_residual_scale"], k=cfg["k"] if r == "token_topk" else 0,
+             idx=sel if r == "token_topk" else None, w=w if r == "token_topk" else None)
+    if r == "expert_choice":
+        m.select_expert_choice(probs, cfg["group_size"], cfg["capacity"], sel, w)
+    ws = m.alloc_workspace(c, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    offsets = torch.empty(c.n_heavy + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(na, dtype=torch.int32, device=dev)
+    row_of = torch.empty(na, dtype=torch.int32, device=dev)
+    ec = r == "expert_choice"
+    tok_ptr = torch.empty(T + 1, dtype=torch.int32, device=dev) if ec else None
+    tok_assign = torch.empty(na, dtype=torch.int32, device=dev) if ec else None
+    x_perm = torch.empty(na, d, dtype=inp["x"].dtype, device=dev)
+    m.dispatch(c, sel, inp["x"], x_perm, offsets, perm, row_of, tok_ptr, tok_assign, status, ws)
+    y_perm = torch.empty(na, d, dtype=inp["x"].dtype, device=dev)
+    y_sh = torch.empty(T, d, dtype=inp["x"].dtype, device=dev) if cfg["n_shared"] else None
+    m.grouped_mlp(c, x_perm, offsets, inp["W1"], inp["W2"], inp["x"], inp["Ws1"], inp["Ws2"],
+                  y_perm, y_sh, status, ws)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    off = offsets.cpu().numpy()
+    pm = perm.cpu().numpy()
+    x_h = gen.to_numpy_f32(inp["x"])
+    rng = np.random.default_rng(99)
+    # four experts: the first, the last and the two with the most / fewest rows
+    cnt = np.diff(off)
+    live = np.nonzero(cnt > 0)[0]
+    experts = sorted({int(live[0]), int(live[-1]), int(live[np.argmax(cnt[live])]),
+                      int(live[np.argmin(cnt[live])])})
+    for e in experts:
+        rows = _sample_rows(int(off[e]), int(off[e + 1]), 64, rng)
+        W1e = gen.to_numpy_f32(inp["W1"][e])
+        W2e = gen.to_numpy_f32(inp["W2"][e])
+        ref = oracle.heavy_expert(cfg["act"], x_h[pm[rows]], W1e, W2e, cfg["h"])
+        got = gen.to_numpy_f32(y_perm[torch.as_tensor(rows, device=dev).long()])
+        err = H.normwise(got, ref)
+        H.log_errors(f"grouped_mlp/{name}/expert{e}", err, err)
+        assert err <= H.Y_TOL[cfg["dtype"]], (e, err)
+    if y_sh is not None:
+        tokens = _sample_rows(0, T, 128, rng)
+        ref = oracle.mlp_gelu(x_h[tokens], gen.to_numpy_f32(inp["Ws1"]),
+                              gen.to_numpy_f32(inp["Ws2"]))
+        got = gen.to_numpy_f32(y_sh[torch.as_tensor(tokens, device=dev).long()])
+        err = H.normwise(got, ref)
+        H.log_errors(f"grouped_mlp/{name}/shared", err, err)
+        assert err <= H.Y_TOL[cfg["dtype"]], err
 
 
 # ---------------------------------------------------------------- edge cases
@@ -293,8 +462,7 @@ def test_edge_cases(label, name, over):
     hin = H.host(inp)
     _check_router(cfg, hin, out)
     sel = _check_selection(cfg, out)
-    y_ref = H.oracle_layer(cfg, hin, sel)
-    assert H.normwise(out["y"], y_ref) <= H.Y_TOL[cfg["dtype"]]
+    H.log_errors(f"edge/{label}", *H.check_layer_outputs(cfg, inp, hin, sel, out))
     if label == "all_zero_compute":
         assert int(out["offsets"][-1]) == 0  # no heavy rows: no GEMM tiles at all
 
