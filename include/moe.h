@@ -75,6 +75,8 @@ enum moe_status {
 #define MOE_DEV_BAD_TOKEN 2u  /* a selected token id outside [0, T) */
 #define MOE_DEV_TIMEOUT 4u    /* a bounded wait inside a kernel expired */
 #define MOE_DEV_OVERFLOW 8u   /* more rows than the caller's buffers hold */
+#define MOE_DEV_BAD_INDEX 16u /* MOE_DEBUG builds: a caller-supplied row offset, row or
+                                 token-list index out of range (skipped) */
 
 enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 };
 enum moe_routing { MOE_TOKEN_TOPK = 0, MOE_EXPERT_CHOICE = 1, MOE_DES_VOTE = 2, MOE_DES_SEQ = 3 };
@@ -351,6 +353,18 @@ MOE_API int moe_combine(const moe_config *cfg, const void *y_perm,
  */
 MOE_API int moe_activation(const float *x, float *y, int64_t n, int act,
                            moe_stream_t stream);
+
+/*
+ * How this copy of the library was built (no counterpart on the pages):
+ * MOE_BUILD_DEBUG is set in the MOE_DEBUG build (libmoe_debug.so), whose
+ * kernels also range-check the row offsets, rows and token lists that a
+ * caller hands to moe_grouped_mlp and moe_combine: an index out of range
+ * sets MOE_DEV_BAD_INDEX in dev_status and its group, slot or token is
+ * skipped, where the regular build (which trusts those arrays, as
+ * moe_dispatch writes them) could read or write out of bounds.
+ */
+#define MOE_BUILD_DEBUG 1
+MOE_API int moe_build_flags(void);
 
 /*
  * Test hook for failure detection (no counterpart on the pages). Blocks of

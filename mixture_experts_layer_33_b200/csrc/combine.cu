@@ -99,8 +99,20 @@ __device__ __forceinline__ void slot_meta(const CombineArgs &a, const KindTable 
   wgt = 0.f;
   mix = false;
   const int asg = ec ? a.tok_assign[j] : j;
+#if MOE_DEBUG
+  if (asg < 0 || asg >= a.y_rows) {  // a token list entry out of range: skip the slot
+    set_status(a.dev_status, MOE_DEV_BAD_INDEX);
+    return;
+  }
+#endif
   const int e = ec ? (int)((asg / a.C) % a.E) : a.sel[asg];
-  const int row = a.row_of[asg];
+  int row = a.row_of[asg];
+#if MOE_DEBUG
+  if (row >= a.y_rows) {  // a row past the expert outputs: no term
+    set_status(a.dev_status, MOE_DEV_BAD_INDEX);
+    row = -1;
+  }
+#endif
   const float wv = a.w[asg];
   if (e >= 0 && e < a.E) {
     const int kind = kinds.kind[e];
@@ -165,6 +177,12 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(CombineArgs a, KindTa
     int a0, a1;
     if (ec) { a0 = a.tok_ptr[s]; a1 = a.tok_ptr[s + 1]; }
     else { a0 = s * a.k; a1 = a0 + a.k; }
+#if MOE_DEBUG
+    if (a0 < 0 || a1 < a0 || a1 > a.y_rows) {  // a token list out of range: no slots
+      if (lane == 0) set_status(a.dev_status, MOE_DEV_BAD_INDEX);
+      a0 = a1 = 0;
+    }
+#endif
     const bool one_group = a1 - a0 <= 32;
     // Slot metadata (and the coefficient of x_s from mixed constant
     // experts) once per token; a token with more than 32 slots re-reads

@@ -27,6 +27,28 @@ __device__ __forceinline__ void set_status(int32_t *st, uint32_t bits) {
   if (st) atomicOr(reinterpret_cast<unsigned int *>(st), bits);
 }
 
+// MOE_DEBUG builds range-check indices that callers hand in (row offsets,
+// rows, token lists); other builds trust them (moe_dispatch writes them).
+#ifndef MOE_DEBUG
+#define MOE_DEBUG 0
+#endif
+
+// The rows [lo, hi) of a group read from caller offsets: in MOE_DEBUG
+// builds a group outside 0 <= lo <= hi <= rows, or with more than max_cnt
+// rows, is flagged (MOE_DEV_BAD_INDEX) and treated as empty.
+template <typename I>
+__device__ __forceinline__ void check_group_rows(I &lo, I &hi, int64_t rows, int32_t *status,
+                                                 int64_t max_cnt = INT64_MAX) {
+#if MOE_DEBUG
+  if (lo < 0 || hi < lo || (int64_t)hi > rows || (int64_t)(hi - lo) > max_cnt) {
+    set_status(status, MOE_DEV_BAD_INDEX);
+    lo = hi = 0;
+  }
+#else
+  (void)lo; (void)hi; (void)rows; (void)status; (void)max_cnt;
+#endif
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

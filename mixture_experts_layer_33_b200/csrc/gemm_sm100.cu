@@ -268,6 +268,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
         if (g < pr.n_groups) {
           lo = pr.offsets ? pr.offsets[g] : 0;
           hi = pr.offsets ? pr.offsets[g + 1] : (int)pr.a_rows;
+          check_group_rows(lo, hi, pr.a_rows, p.status);
         }
         int tiles = (g < pr.n_groups && hi > lo) ? ((hi - lo + BM - 1) / BM) * ntn : 0;
         int inc = warp_inclusive_scan(tiles);
@@ -502,6 +503,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
         if (g < pr.n_groups) {
           lo = pr.offsets ? pr.offsets[g] : 0;
           hi = pr.offsets ? pr.offsets[g + 1] : (int)pr.a_rows;
+          check_group_rows(lo, hi, pr.a_rows, p.status);
         }
         int tiles = (g < pr.n_groups && hi > lo) ? ((hi - lo + BMP - 1) / BMP) * ntn : 0;
         int inc = warp_inclusive_scan(tiles);

@@ -204,6 +204,7 @@ struct GemmProblem {
   int64_t ld_out;
   const void *residual; // optional [rows, ld_res] bf16 added before the output is rounded
   int64_t ld_res;
+  int32_t *status;      // device status word for MOE_DEBUG range checks (fp32 path), nullable
 };
 
 // Upper bound of the m-tiles of height bm over all groups of a problem.
@@ -247,6 +248,7 @@ struct CombineArgs {
   const void *x, *const_vecs, *residual;
   void *y;
   int32_t *dev_status;
+  int64_t y_rows;  // rows of y_perm (= assignments): the range MOE_DEBUG builds check rows against
 };
 int launch_combine(const CombineArgs &a, const KindTable &kinds,
                    cudaStream_t stream);

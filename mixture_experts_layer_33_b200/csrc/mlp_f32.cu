@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(kThreads) grouped_gemm_f32_kernel(GemmProblem 
     for (int gi = 0; gi < p.n_groups; ++gi) {
       int64_t lo = p.offsets ? p.offsets[gi] : 0;
       int64_t hi = p.offsets ? p.offsets[gi + 1] : p.a_rows;
+      check_group_rows(lo, hi, p.a_rows, p.status);
       int64_t mt = (hi - lo + kBM - 1) / kBM;
       if (t < mt) { g = gi; r0 = (int)(lo + t * kBM); r1 = (int)hi; break; }
       t -= mt;

@@ -4,6 +4,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -273,6 +275,7 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
   g2s.A = H_sh; g2s.a_rows = c.T; g2s.B = Ws2; g2s.n_groups = 1; g2s.offsets = nullptr;
   g2s.N = c.d; g2s.b_rows_per_group = c.d; g2s.K = (int)hs; g2s.out = y_shared; g2s.ld_out = c.d;
   g2s.residual = shared_residual; g2s.ld_res = c.d;
+  g1r.status = g1s.status = g2r.status = g2s.status = dev_status;
   const bool routed = c.n_heavy > 0 && na > 0;
   const bool shared = hs > 0 && c.T > 0;
 
@@ -345,8 +348,30 @@ CombineArgs combine_args(const moe_config &c, const void *y_perm, const void *y_
   a.y_perm = y_perm; a.y_shared = y_shared; a.sel = sel; a.w = w; a.row_of = row_of;
   a.tok_ptr = tok_ptr; a.tok_assign = tok_assign; a.x = x; a.const_vecs = const_vecs;
   a.residual = residual; a.y = y; a.dev_status = dev_status;
+  a.y_rows = n_assign_of(c);
   return a;
 }
+
+// NVTX range over a scope: names the layer's stages for a profiler
+// (header-only NVTX; a no-op unless a tool is attached).
+struct NvtxScope {
+  explicit NvtxScope(const char *name) { nvtxRangePushA(name); }
+  ~NvtxScope() { nvtxRangePop(); }
+  NvtxScope(const NvtxScope &) = delete;
+  NvtxScope &operator=(const NvtxScope &) = delete;
+};
+// Consecutive NVTX ranges: next() closes the open one and opens another.
+struct NvtxStages {
+  bool open = false;
+  void next(const char *name) {
+    if (open) nvtxRangePop();
+    nvtxRangePushA(name);
+    open = true;
+  }
+  ~NvtxStages() {
+    if (open) nvtxRangePop();
+  }
+};
 
 int forward_device(const moe_config &c, const void *x, const void *residual,
                    const float *z_prev, const void *W_r, const float *bias, const void *W1,
@@ -367,12 +392,14 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
   void *Y = at<void>(ws, L.Y);
   void *Y_sh = hs ? at<void>(ws, L.Y_sh) : nullptr;
   void *x_perm = at<void>(ws, L.x_perm);
+  NvtxScope layer_range("moe_forward");
 
   int st = MOE_OK;
   const int n_part = router_split_parts(c.T, c.d, c.dtype);
   const bool streaming = c.dtype == MOE_BF16 && stream_mlp_supported(c.T);
   bool routed_and_gathered = false;
   if (small_f32_supported(c)) {
+    NvtxScope r("moe_forward/one_launch_f32");
     // Small fp32 token-choice layer without a shared expert: the whole layer
     // in one launch, a CTA per token (its per-expert row counts, and the
     // CTA counter that finds the last CTA, start at zero).
@@ -391,6 +418,7 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
     return launch_small_f32(fa, kind_table(c), stream);
   }
   if (moe_block_supported(c)) {
+    NvtxScope r("moe_forward/one_launch_block");
     // Small bf16 block without a shared expert: the whole layer in one
     // persistent kernel (router K-sliced over the CTAs, selection, a weight
     // stream that starts as soon as the experts to stream are known, the
@@ -413,6 +441,8 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
     ba.dev_status = dev_status;
     return launch_moe_block(ba, kind_table(c), W1, W2, c.act, stream);
   }
+  NvtxStages stage;
+  stage.next("moe_forward/route");
   if (n_part > 0 && small_route_supported(c.T, c.E, c.k, c.routing, c.dtype)) {
     // Small bf16 block (<= 128 tokens): the router split over the model
     // width, then one cooperative kernel finishes the router, selects (DES:
@@ -468,6 +498,7 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
                           reinterpret_cast<int32_t *>(at<int64_t>(ws, L.votes)), sel, w, stream);
     if (st != MOE_OK) return st;
   }
+  stage.next("moe_forward/dispatch");
   if (!routed_and_gathered) {
     DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
     if (streaming) {  // the dispatch clears the weight-streaming kernel's counters
@@ -490,12 +521,14 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
   // writes y = residual + shared(x) straight into y, and the combine then adds
   // the routed terms in place (no shared-output buffer round trip).
   const bool shared_into_y = hs > 0 && c.dtype == MOE_BF16 && !streaming && c.T > 0;
+  stage.next("moe_forward/grouped_mlp");
   st = run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, Y, shared_into_y ? y : Y_sh,
                        dev_status, ws, L, stream, streaming, shared_into_y ? residual : nullptr);
   if (st != MOE_OK) return st;
   CombineArgs ca = combine_args(c, Y, shared_into_y ? nullptr : Y_sh, sel, w, row_of, tok_ptr,
                                 tok_assign, x, const_vecs, shared_into_y ? y : residual, y,
                                 dev_status);
+  stage.next("moe_forward/combine");
   return launch_combine(ca, kind_table(c), stream);
 }
 
@@ -687,6 +720,8 @@ int moe_activation(const float *x, float *y, int64_t n, int act, moe_stream_t st
   if (n > 0 && (!x || !y)) return MOE_ERR_INVALID_ARG;
   return launch_activation(x, y, n, act, stream);
 }
+
+int moe_build_flags(void) { return MOE_DEBUG ? MOE_BUILD_DEBUG : 0; }
 
 int moe_test_set_barrier_wait(uint64_t limit_ns, int extra_arrivals) {
   if (limit_ns > 2000000000ull || extra_arrivals < 0 || extra_arrivals > 1024)

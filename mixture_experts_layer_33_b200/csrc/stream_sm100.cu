@@ -165,6 +165,7 @@ expert_stream_kernel(const __grid_constant__ CUtensorMap tmW1, const __grid_cons
         if (g < p.n_groups) {
           lo = p.offsets ? p.offsets[g] : 0;
           hi = p.offsets ? p.offsets[g + 1] : p.t_rows;
+          check_group_rows(lo, hi, p.t_rows, p.status, NB);  // a group spans <= NB token columns
         }
         const int n = (g < p.n_groups && hi > lo) ? blocks : 0;
         const int inc = warp_inclusive_scan(n);

@@ -5,6 +5,9 @@ CUDA kernels. PyTorch supplies device memory and the current stream.
 Importing this module loads the library and raises ImportError if it has
 not been built (``python -m mixture_experts_layer_33_b200.build``); calls
 raise RuntimeError with the library's status string when a call fails.
+With MOE_DEBUG=1 in the environment it loads the MOE_DEBUG build
+(``libmoe_debug.so``, ``build --debug``) instead: the same entry points,
+whose kernels also range-check the indices callers hand in.
 """
 
 from __future__ import annotations
@@ -14,14 +17,17 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+DEBUG_BUILD = os.environ.get("MOE_DEBUG", "0") == "1"
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libmoe_debug.so" if DEBUG_BUILD else "libmoe.so")
 
 MOE_OK = 0
 F32, BF16 = 0, 1
 TOKEN_TOPK, EXPERT_CHOICE, DES_VOTE, DES_SEQ = 0, 1, 2, 3
 GELU_ERF, SWIGLU = 0, 1
 HEAVY, IDENTITY, ZERO, CONST = 0, 1, 2, 3
-DEV_BAD_EXPERT, DEV_BAD_TOKEN, DEV_TIMEOUT, DEV_OVERFLOW = 1, 2, 4, 8
+DEV_BAD_EXPERT, DEV_BAD_TOKEN, DEV_TIMEOUT, DEV_OVERFLOW, DEV_BAD_INDEX = 1, 2, 4, 8, 16
+BUILD_DEBUG = 1  # moe_build_flags() bit of the MOE_DEBUG build
 MAX_EXPERTS = 256
 
 # Names of every entry point include/moe.h declares.
@@ -30,7 +36,7 @@ ENTRY_POINTS = (
     "moe_workspace_size", "moe_router", "moe_select_topk",
     "moe_select_expert_choice", "moe_core_set_vote", "moe_core_set_union", "moe_dispatch",
     "moe_grouped_mlp", "moe_combine", "moe_forward", "moe_forward_host",
-    "moe_dispatch_noalloc", "moe_activation", "moe_test_set_barrier_wait",
+    "moe_dispatch_noalloc", "moe_activation", "moe_test_set_barrier_wait", "moe_build_flags",
 )
 NOALLOC_SCRATCH_BYTES = 256 * 1024  # MOE_NOALLOC_SCRATCH_BYTES
 
@@ -70,6 +76,7 @@ _SIGS = {
     "moe_dispatch_noalloc": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_activation": (_i32, [_vp, _vp, ctypes.c_int64, _i32, _vp]),
     "moe_test_set_barrier_wait": (_i32, [ctypes.c_uint64, _i32]),
+    "moe_build_flags": (_i32, []),
     "moe_grouped_mlp": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                _vp]),
     "moe_combine": (_i32, [_CFG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -95,6 +102,11 @@ def _load():
 
 LIB = _load()
 LIB_PATH = _LIB_PATH
+
+
+def build_flags():
+    """MOE_BUILD_* bits of the loaded library (BUILD_DEBUG: the MOE_DEBUG build)."""
+    return LIB.moe_build_flags()
 
 
 def status_string(code):

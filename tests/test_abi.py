@@ -131,3 +131,16 @@ def test_barrier_wait_hook_checks_its_arguments(m):
     assert m.LIB.moe_test_set_barrier_wait(0, 1025) == 1
     assert m.LIB.moe_test_set_barrier_wait(1000, 1) == 0
     assert m.LIB.moe_test_set_barrier_wait(0, 0) == 0
+
+
+def test_debug_build_exports_the_same_symbols_and_says_so(m):
+    """The MOE_DEBUG variant exports every declared entry point and reports
+    itself through moe_build_flags; the regular build does not."""
+    from mixture_experts_layer_33_b200 import build
+    path = build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(dbg, name), name
+    dbg.moe_build_flags.restype = ctypes.c_int
+    assert dbg.moe_build_flags() & m.BUILD_DEBUG
+    assert not m.build_flags() & m.BUILD_DEBUG

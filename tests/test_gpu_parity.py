@@ -404,6 +404,9 @@ EDGE = [
     # (N = 1024, expert choice)
     ("gemm2_pair_two_mma_384", "ditmoe_xl", dict(T=3000, d=768, h=2048, h_shared=2048)),
     ("gemm2_pair_two_mma_512", "ecdit", dict(T=16 * 128, group_size=128, d=1024, E=8, h=2048, capacity=32)),
+    # 160 wide (256 x 512) down-projection tiles over 74 CTA pairs: a last
+    # wave of 12 tiles on a grid of many pairs
+    ("ec_wide_partial_wave", "ecdit", dict(T=40 * 128, group_size=128, d=1024, E=16, h=2048, capacity=32)),
     ("all_zero_compute", "mmoe", dict(T=200, d=128, h=256, h_shared=128, zero_compute_logit_bias=60.0)),
     ("ec_full_capacity", "ecdit", dict(T=64, group_size=16, d=128, E=4, h=256, capacity=16)),
     ("ec_whole_batch", "ecdit", dict(T=2048, group_size=2048, d=128, E=8, h=256, capacity=512)),
