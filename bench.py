@@ -57,12 +57,12 @@ class L2Flush:
 NCU_TRAFFIC = {
     "des_vote": {"bytes": (421.61 + 4.33) * 1e6,
                  "source": "block_sm100.cu", "sha256_16": "62215f5b9bfc055a"},
-    "ditmoe_xl": {"bytes": (162.94 + 258.17 + 459.52 + 38.40) * 1e6,
-                  "source": "gemm_sm100.cu", "sha256_16": "cfc640b5c5107701"},
-    "ecdit": {"bytes": (1256.95 + 252.12 + 1474.95 + 58.29) * 1e6,
-              "source": "gemm_sm100.cu", "sha256_16": "cfc640b5c5107701"},
-    "mmoe": {"bytes": (231.67 + 155.34 + 421.20 + 40.03) * 1e6,
-             "source": "gemm_sm100.cu", "sha256_16": "cfc640b5c5107701"},
+    "ditmoe_xl": {"bytes": (162.95 + 258.21 + 459.16 + 39.03) * 1e6,
+                  "source": "gemm_sm100.cu", "sha256_16": "b9a034e2f1d79c8b"},
+    "ecdit": {"bytes": (1288.91 + 252.81 + 1576.19 + 58.56) * 1e6,
+              "source": "gemm_sm100.cu", "sha256_16": "b9a034e2f1d79c8b"},
+    "mmoe": {"bytes": (231.53 + 155.17 + 421.38 + 40.33) * 1e6,
+             "source": "gemm_sm100.cu", "sha256_16": "b9a034e2f1d79c8b"},
 }
 
 
