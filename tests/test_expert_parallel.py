@@ -17,7 +17,7 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from mixture_experts_layer_33_b200.expert_parallel import (ExpertShard, InterweavedEP, ep_forward,
-                                                           exchange_plan)
+                                                           exchange_plan, merge_stale_slots)
 from oracle import moe_oracle as om
 
 H, I, Z, C = om.HEAVY, om.IDENTITY, om.ZERO, om.CONST
@@ -295,3 +295,21 @@ def test_cuda_steps_take_token_choice_only():
     for name in ("ecdit", "des_vote"):
         with pytest.raises(ValueError):
             CudaOps(gen.workload(name), ExpertShard(4, 2), 0, None, None, None, device="cpu")
+
+
+def test_merge_stale_slots_keeps_previous_heavy_and_current_light_slots():
+    # 3 tokens, k = 2, experts 0..3 heavy, 4..5 zero-computation; -1 empty.
+    prev_sel = torch.tensor([0, 4, 5, 3, -1, 2], dtype=torch.int32)
+    prev_w = torch.tensor([.1, .2, .3, .4, .5, .6])
+    prev_row = np.array([7, -1, -1, 9, -1, 4], dtype=np.int32)
+    sel = torch.tensor([4, 1, 2, 3, 5, 0], dtype=torch.int32)
+    w = torch.tensor([.7, .8, .9, 1.0, 1.1, 1.2])
+    m_sel, m_w, m_row = merge_stale_slots(prev_sel, prev_w, prev_row, sel, w, 4, 2)
+    # per token: [prev slot 0, prev slot 1, current slot 0, current slot 1]
+    assert m_sel.tolist() == [0, -1, 4, -1,
+                              -1, 3, -1, -1,
+                              -1, 2, 5, -1]
+    assert m_row.tolist() == [7, -1, -1, -1,
+                              -1, 9, -1, -1,
+                              -1, 4, -1, -1]
+    np.testing.assert_allclose(m_w.numpy(), [.1, .2, .7, .8, .3, .4, .9, 1.0, .5, .6, 1.1, 1.2])

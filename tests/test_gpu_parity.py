@@ -470,6 +470,36 @@ def test_edge_cases(label, name, over):
         assert int(out["offsets"][-1]) == 0  # no heavy rows: no GEMM tiles at all
 
 
+# The library's limits and ragged widths, sampled like the full workloads:
+# the largest DES block (4096 tokens), the largest expert-choice group
+# (16384 tokens, one group), 128 experts under top-8 over 65536 tokens
+# (half a million assignments, 512 dispatch blocks), and model / hidden
+# widths that are not multiples of the 64-wide K block (K = 200 and 168:
+# the last TMA box of every row is partly past the end and zero-filled).
+LIMITS = [
+    ("des_block_4096", "des_vote", dict(T=4096, d=256, h=128)),
+    ("ec_group_16384", "ecdit", dict(T=16384, group_size=16384, d=128, E=8, h=256, capacity=2048)),
+    ("topk_E128_T65536", "ditmoe_xl", dict(T=65536, d=128, E=128, k=8, h=128, n_shared=0)),
+    ("ragged_K_200_168", "mmoe", dict(T=1000, d=200, h=168, h_shared=168)),
+]
+
+
+@pytest.mark.parametrize("label,name,over", LIMITS, ids=[c[0] for c in LIMITS])
+def test_limits_and_ragged_widths_sampled(label, name, over):
+    cfg = gen.workload(name, **over)
+    inp = gen.make_inputs(cfg, "cuda")
+    out = H.run_layer(cfg, inp)
+    assert out["status"] == 0
+    hin = H.host(inp)
+    _check_router(cfg, hin, out)
+    sel = _check_selection(cfg, out)
+    rng = np.random.default_rng(4321)
+    T = cfg["T"]
+    tokens = np.sort(rng.choice(T, size=min(T, 256), replace=False))
+    tokens[0], tokens[-1] = 0, T - 1
+    H.log_errors(f"limits/{label}", *H.check_layer_outputs(cfg, inp, hin, sel, out, tokens=tokens))
+
+
 @pytest.mark.parametrize("N,kl", [(32, 2), (1, 2), (64, 1), (300, 3)])
 def test_core_set_union_entry_point(N, kl):
     """moe_core_set_union against the oracle's DES-Seq on the GPU's own probabilities."""
