@@ -33,11 +33,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait. Returns false if the kernel is aborting (another role gave
-// up) or this wait expired (then it raises the abort itself).
-static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       int32_t *status, bool watch_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
+// The bounded wait's slow path, out of line: spin, watching the abort flag
+// and the time limit.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                                   volatile int *abort_flag, int32_t *status,
+                                                   bool watch_abort) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -50,6 +50,16 @@ static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, vol
       }
     }
   }
+}
+// Bounded wait. Returns false if the kernel is aborting (another role gave
+// up) or this wait expired (then it raises the abort itself). The check of
+// an already completed phase is inline: a call per wait on the tensor
+// pipelines' hot loops (every k-block) cost the grouped GEMMs ~5 % of their
+// time.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          int32_t *status, bool watch_abort = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, status, watch_abort);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
@@ -167,11 +177,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "memory");
   return ok != 0;
 }
-// Bounded wait with cluster-scope acquire (arrivals may come from the peer CTA).
-static __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
-                                                       volatile int *abort_flag, int32_t *status,
-                                                       bool watch_abort = true) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+// Bounded wait with cluster-scope acquire (arrivals may come from the peer
+// CTA): the slow path out of line, the completed-phase check inline.
+static __device__ __noinline__ bool mbar_wait_cluster_slow(uint32_t bar, uint32_t parity,
+                                                           volatile int *abort_flag, int32_t *status,
+                                                           bool watch_abort) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t spin = 1;; ++spin) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
@@ -184,6 +194,12 @@ static __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t par
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  volatile int *abort_flag, int32_t *status,
+                                                  bool watch_abort = true) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  return mbar_wait_cluster_slow(bar, parity, abort_flag, status, watch_abort);
 }
 // TMA tile load into this CTA's shared memory whose completion is counted on
 // an mbarrier that may be in the peer CTA (the pair's leader).
