@@ -45,7 +45,8 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle atom row
 constexpr int kEpiWarps = 8;                    // two per TMEM lane quadrant
 constexpr int kThreads = 64 + 32 * kEpiWarps;   // producer warp, MMA warp, epilogue warps
-constexpr int kMaxEntries = 2 * MOE_MAX_EXPERTS + 2;
+constexpr int kMaxEntries = 2 * kMaxLayerExperts + 2;  // (problem, group) entries of a launch
+constexpr uint32_t kStageOutBytes = 32 * 32 * 2;           // an epilogue warp's 32 x 32 bf16 staging tile
 
 struct ProbDev {
   const int32_t *offsets;
@@ -58,6 +59,7 @@ struct ProbDev {
   int vec32;  // rows of `out` start on 32-byte boundaries: 256-bit stores
   const __nv_bfloat16 *residual;  // optional, added before rounding (bf16 outputs)
   int64_t ld_res;
+  int tma_out;  // bf16 output stored by TMA from shared-memory staging tiles (one-SM kernel)
 };
 struct ParamsDev {
   int n_probs;
@@ -206,10 +208,53 @@ __device__ __forceinline__ void store_row32(const ProbDev &pr, int row, int col,
   }
 }
 
+// 32 consecutive output columns of this lane's row as bf16 (residual added
+// before rounding), written as row `lane` of the warp's 32 x 32 staging tile
+// in the TMA 64-byte swizzle: 16-byte chunk q of row r lands at chunk
+// q ^ ((r >> 1) & 3), so the 32 lanes' 16-byte writes spread over all banks.
+// Columns past N are staged as zero and clipped by the TMA store.
+__device__ __forceinline__ void stage_row32_bf16(const ProbDev &pr, int row, int col, const float (&v)[32],
+                                                 uint32_t stg, int lane) {
+  float r[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = 0.f;
+  const bool full = col + 32 <= pr.N;
+  if (pr.residual) {
+    const __nv_bfloat16 *rp = pr.residual + (int64_t)row * pr.ld_res + col;
+    if (full) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        float t[8];
+        load8(rp + i, t);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[i + j] = t[j];
+      }
+    } else {
+      for (int i = 0; i < 32 && col + i < pr.N; ++i) r[i] = __bfloat162float(rp[i]);
+    }
+  }
+  uint32_t w[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const bool in = full || col + 2 * j < pr.N;
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(in ? v[2 * j] + r[2 * j] : 0.f,
+                                              in ? v[2 * j + 1] + r[2 * j + 1] : 0.f);
+    w[j] = *reinterpret_cast<uint32_t *>(&h2);
+  }
+  const uint32_t rowaddr = stg + (uint32_t)lane * 64u;
+  const uint32_t sw = (uint32_t)((lane >> 1) & 3);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowaddr + (((uint32_t)q ^ sw) << 4)),
+                 "r"(w[4 * q]), "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                 : "memory");
+}
+
 template <int BN, int ACT, bool OUT_F32, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                       const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                        const ParamsDev p) {
   constexpr int BNO = (ACT == kActSwiglu) ? BN / 2 : BN;  // output columns per tile
   constexpr uint32_t A_BYTES = BM * BK * 2;
@@ -229,6 +274,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
                                               ~(uintptr_t)1023);
   const uint32_t sA = smem_u32(base);
   const uint32_t sB = sA + STAGES * A_BYTES;
+  const uint32_t sO = sB + STAGES * B_BYTES;  // the epilogue warps' staging tiles
   const uint32_t full0 = smem_u32(&bars[0]);
   const uint32_t empty0 = smem_u32(&bars[STAGES]);
   const uint32_t tfull0 = smem_u32(&bars[2 * STAGES]);
@@ -371,6 +417,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
     const int quad = warp & 3;                  // TMEM lanes this warp may read
     const int lrow = quad * 32 + lane;
     const int c_lo = ((warp - 2) / 4) * (BNO / 2);  // this warp's half of the columns
+    const uint32_t stg = sO + (uint32_t)(warp - 2) * kStageOutBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
@@ -382,6 +429,12 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
       const int row = sched.row0[e] + mt * BM + lrow;
       const bool valid = row < sched.row_end[e];
       const int col0 = nt * BNO;
+      // Whole 32-row blocks of the group go out as TMA tile stores; a block
+      // reaching past the group's last row (whose next rows belong to the
+      // next group) keeps per-lane stores of its valid rows.
+      const int wrow0 = sched.row0[e] + mt * BM + quad * 32;
+      const bool tma_rows = !OUT_F32 && pr.tma_out && wrow0 + 32 <= sched.row_end[e];
+      const CUtensorMap *mO = sched.prob[e] ? &tmO1 : &tmO0;
       // Warp-uniform: tcgen05.ld below is .sync.aligned, so either every
       // lane proceeds or every lane leaves.
       const bool ready = mbar_wait(tfull0 + 8 * acc, acc_phase, &abort_flag, p.status);
@@ -401,13 +454,26 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_co
 #pragma unroll
           for (int i = 0; i < 32; i += 2) gelu_erf_x2(v[i], v[i + 1]);
         }
-        if (valid) store_row32<OUT_F32>(pr, row, col0 + c, v);
+        if (tma_rows) {
+          if (lane == 0) bulk_wait_read_all();  // the tile's previous store has read it
+          __syncwarp();
+          stage_row32_bf16(pr, row, col0 + c, v, stg, lane);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(mO, col0 + c, wrow0, stg);
+            bulk_commit();
+          }
+        } else if (valid) {
+          store_row32<OUT_F32>(pr, row, col0 + c, v);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait_all();  // every tile store has landed before the CTA exits
   }
 
   tc_fence_before();
@@ -696,6 +762,24 @@ bool make_map(CUtensorMap *m, const void *ptr, int64_t rows, int64_t cols, int b
   return r == CUDA_SUCCESS;
 }
 
+// bf16 output [rows, N] with row stride ld_out, box of 32 x 32 staged with the
+// 64-byte swizzle. False when the output cannot take TMA stores (a base off
+// 16 bytes or a row stride that is not a multiple of 16 bytes).
+bool make_out_map(CUtensorMap *m, const GemmProblem &q) {
+  if ((reinterpret_cast<uintptr_t>(q.out) & 15u) != 0 || (q.ld_out * 2) % 16 != 0 || q.a_rows <= 0)
+    return false;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)q.N, (cuuint64_t)q.a_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)q.ld_out * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q.out, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool vec32_ok(const GemmProblem &q, int elem) {
   return (reinterpret_cast<uintptr_t>(q.out) & 31u) == 0 && (q.ld_out * elem) % 32 == 0;
 }
@@ -705,10 +789,11 @@ int run_tc(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t 
   constexpr uint32_t STAGE_BYTES = (BM + BN) * BK * 2;
   constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
   constexpr int BNO = (ACT == kActSwiglu) ? BN / 2 : BN;
-  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES;
+  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + (OUT_F32 ? 0 : kEpiWarps * kStageOutBytes);
 
-  CUtensorMap maps[4];
+  CUtensorMap maps[4], omaps[2];
   memset(maps, 0, sizeof(maps));
+  memset(omaps, 0, sizeof(omaps));
   ParamsDev pd;
   memset(&pd, 0, sizeof(pd));
   pd.n_probs = n_probs;
@@ -730,15 +815,16 @@ int run_tc(const GemmProblem *probs, int n_probs, int32_t *status, cudaStream_t 
     pd.pr[i].vec32 = vec32_ok(q, OUT_F32 ? 4 : 2);
     pd.pr[i].residual = static_cast<const __nv_bfloat16 *>(q.residual);
     pd.pr[i].ld_res = q.ld_res;
+    pd.pr[i].tma_out = !OUT_F32 && make_out_map(&omaps[i], q);
     max_tiles += max_m_tiles(q, BM) * ((q.N + BNO - 1) / BNO);
   }
-  if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; }
+  if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; omaps[1] = omaps[0]; }
   if (max_tiles == 0) return MOE_OK;
   auto kern = grouped_gemm_tc_kernel<BN, ACT, OUT_F32, STAGES>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)max_tiles;
-  kern<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], pd);
+  kern<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], omaps[0], omaps[1], pd);
   return last_launch_status();
 }
 

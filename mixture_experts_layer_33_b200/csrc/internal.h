@@ -20,6 +20,10 @@ struct KindTable;
     if (moe_err_ != cudaSuccess) return MOE_ERR_CUDA;        \
   } while (0)
 
+// Experts per layer the library takes (moe_config.E; larger is
+// MOE_ERR_UNSUPPORTED).
+constexpr int kMaxLayerExperts = 128;
+
 inline int last_launch_status() {
   return cudaPeekAtLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -34,7 +34,8 @@ int check_config(const moe_config *c) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_BF16 && c->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
   if (c->T < 0 || c->d < 8 || c->d % 8 != 0) return MOE_ERR_INVALID_ARG;
-  if (c->E < 1 || c->E > 128) return c->E > 128 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  if (c->E < 1 || c->E > kMaxLayerExperts)
+    return c->E > kMaxLayerExperts ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
   if (c->n_heavy < 0 || c->n_heavy > c->E) return MOE_ERR_INVALID_ARG;
   if (c->n_heavy > 0 && (c->h < 8 || c->h % 8 != 0)) return MOE_ERR_INVALID_ARG;
   if (c->act != MOE_GELU_ERF && c->act != MOE_SWIGLU) return MOE_ERR_INVALID_ARG;
