@@ -254,11 +254,90 @@ int host_pipe(HostPipe **p) {
   return MOE_OK;
 }
 
+// moe_forward runs the shared expert's up projection (it needs only x) on a
+// per-device side stream while the routed rows are dispatched and gathered
+// on the caller's stream; the down projections wait for both. The stream
+// and its two events are made on first use and kept for the life of the
+// process. A forward holds g_side_mu from the fork's event record to the
+// caller stream's wait on the join, so concurrent callers on one device do
+// not interleave their records and waits.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[kHostMaxDevices];
+
+// Fork of the side stream from a caller's stream, joined back (the caller's
+// stream waits for the side stream's work) by join() or, on an early
+// return, by the destructor, so a captured stream never ends with the side
+// stream unjoined.
+class SideFork {
+ public:
+  explicit SideFork(cudaStream_t stream) : stream_(stream) {}
+  SideFork(const SideFork &) = delete;
+  SideFork &operator=(const SideFork &) = delete;
+  ~SideFork() { join(); }
+  cudaStream_t side() const { return side_->s; }
+  // Work enqueued on side() from here on runs after everything enqueued on
+  // the caller's stream so far.
+  int fork() {
+    int dev = 0;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kHostMaxDevices) return MOE_ERR_UNSUPPORTED;
+    lock_ = std::unique_lock<std::mutex>(g_side_mu);
+    SideStream &ss = g_side[dev];
+    if (!ss.s) {
+      if (!ss.fork) MOE_CUDA_TRY(cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming));
+      if (!ss.join) MOE_CUDA_TRY(cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming));
+      MOE_CUDA_TRY(cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking));  // last: marks it ready
+    }
+    MOE_CUDA_TRY(cudaEventRecord(ss.fork, stream_));
+    MOE_CUDA_TRY(cudaStreamWaitEvent(ss.s, ss.fork, 0));
+    side_ = &ss;
+    return MOE_OK;
+  }
+  // The caller's stream waits for the side stream's work so far.
+  int join() {
+    if (!side_) {
+      if (lock_.owns_lock()) lock_.unlock();
+      return MOE_OK;
+    }
+    SideStream *ss = side_;
+    side_ = nullptr;
+    cudaError_t e = cudaEventRecord(ss->join, ss->s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream_, ss->join, 0);
+    lock_.unlock();
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+
+ private:
+  cudaStream_t stream_;
+  SideStream *side_ = nullptr;
+  std::unique_lock<std::mutex> lock_;
+};
+
+// The shared expert's up projection: H_sh = GELU(x Ws1^T) over all tokens
+// (the shared experts concatenated along the hidden dimension).
+GemmProblem shared_up_problem(const moe_config &c, const void *x, const void *Ws1, void *H_sh,
+                              int32_t *dev_status) {
+  const int64_t hs = (int64_t)c.n_shared * c.h_shared;
+  GemmProblem g{};
+  g.A = x; g.a_rows = c.T; g.B = Ws1; g.n_groups = 1; g.offsets = nullptr;
+  g.N = (int)hs; g.b_rows_per_group = (int)hs; g.K = c.d; g.out = H_sh; g.ld_out = hs;
+  g.status = dev_status;
+  return g;
+}
+
+// `side`: the shared up projection already runs on a forked side stream;
+// the routed up projection runs alone and the down projections wait for
+// the side stream.
 int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offsets,
                     const void *W1, const void *W2, const void *x, const void *Ws1,
                     const void *Ws2, void *y_perm, void *y_shared, int32_t *dev_status,
                     void *ws, const Layout &L, cudaStream_t stream,
-                    bool counters_zeroed = false, const void *shared_residual = nullptr) {
+                    bool counters_zeroed = false, const void *shared_residual = nullptr,
+                    SideFork *side = nullptr) {
   const int64_t na = n_assign_of(c);
   const int64_t hs = (int64_t)c.n_shared * c.h_shared;
   void *H = at<void>(ws, L.H);
@@ -271,8 +350,7 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
   g1r.out = H; g1r.ld_out = c.h;
   g2r.A = H; g2r.a_rows = na; g2r.B = W2; g2r.n_groups = c.n_heavy; g2r.offsets = offsets;
   g2r.N = c.d; g2r.b_rows_per_group = c.d; g2r.K = c.h; g2r.out = y_perm; g2r.ld_out = c.d;
-  g1s.A = x; g1s.a_rows = c.T; g1s.B = Ws1; g1s.n_groups = 1; g1s.offsets = nullptr;
-  g1s.N = (int)hs; g1s.b_rows_per_group = (int)hs; g1s.K = c.d; g1s.out = H_sh; g1s.ld_out = hs;
+  g1s = shared_up_problem(c, x, Ws1, H_sh, dev_status);
   g2s.A = H_sh; g2s.a_rows = c.T; g2s.B = Ws2; g2s.n_groups = 1; g2s.offsets = nullptr;
   g2s.N = c.d; g2s.b_rows_per_group = c.d; g2s.K = (int)hs; g2s.out = y_shared; g2s.ld_out = c.d;
   g2s.residual = shared_residual; g2s.ld_res = c.d;
@@ -294,7 +372,10 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
   }
   if (c.dtype == MOE_BF16) {
     // GEMM1 (+activation): routed and shared in one tile stream when they share the activation.
-    if (routed && shared && act1 == kActGelu) {
+    if (side) {
+      if (routed) st = launch_grouped_gemm_bf16(&g1r, 1, act1, false, dev_status, stream);
+      if (st == MOE_OK) st = side->join();
+    } else if (routed && shared && act1 == kActGelu) {
       GemmProblem p1[2] = {g1r, g1s};
       st = launch_grouped_gemm_bf16(p1, 2, kActGelu, false, dev_status, stream);
     } else {
@@ -499,6 +580,22 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
                           reinterpret_cast<int32_t *>(at<int64_t>(ws, L.votes)), sel, w, stream);
     if (st != MOE_OK) return st;
   }
+  // bf16 grouped-GEMM path with a shared expert: its down-projection epilogue
+  // writes y = residual + shared(x) straight into y, and the combine then adds
+  // the routed terms in place (no shared-output buffer round trip).
+  const bool shared_into_y = hs > 0 && c.dtype == MOE_BF16 && !streaming && c.T > 0;
+  // With routed rows too, the shared up projection runs on the side stream
+  // during the dispatch and row gather (small launches that leave most of
+  // each SM free), joined before the down projections.
+  SideFork side(stream);
+  const bool side_shared = shared_into_y && c.n_heavy > 0 && na > 0 && !routed_and_gathered;
+  if (side_shared) {
+    st = side.fork();
+    if (st != MOE_OK) return st;
+    const GemmProblem g1s = shared_up_problem(c, x, Ws1, at<void>(ws, L.H_sh), dev_status);
+    st = launch_grouped_gemm_bf16(&g1s, 1, kActGelu, false, dev_status, side.side());
+    if (st != MOE_OK) return st;
+  }
   stage.next("moe_forward/dispatch");
   if (!routed_and_gathered) {
     DispatchArgs da = dispatch_args(c, sel, offsets, perm, row_of, tok_ptr, tok_assign, dev_status);
@@ -518,13 +615,10 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
       if (st != MOE_OK) return st;
     }
   }
-  // bf16 grouped-GEMM path with a shared expert: its down-projection epilogue
-  // writes y = residual + shared(x) straight into y, and the combine then adds
-  // the routed terms in place (no shared-output buffer round trip).
-  const bool shared_into_y = hs > 0 && c.dtype == MOE_BF16 && !streaming && c.T > 0;
   stage.next("moe_forward/grouped_mlp");
   st = run_grouped_mlp(c, x_perm, offsets, W1, W2, x, Ws1, Ws2, Y, shared_into_y ? y : Y_sh,
-                       dev_status, ws, L, stream, streaming, shared_into_y ? residual : nullptr);
+                       dev_status, ws, L, stream, streaming, shared_into_y ? residual : nullptr,
+                       side_shared ? &side : nullptr);
   if (st != MOE_OK) return st;
   CombineArgs ca = combine_args(c, Y, shared_into_y ? nullptr : Y_sh, sel, w, row_of, tok_ptr,
                                 tok_assign, x, const_vecs, shared_into_y ? y : residual, y,
