@@ -62,12 +62,12 @@ class L2Flush:
 NCU_TRAFFIC = {
     "des_vote": {"bytes": (421.57 + 4.32) * 1e6,
                  "source": "block_sm100.cu", "sha256_16": "253237819f3ad668"},
-    "ditmoe_xl": {"bytes": (162.97 + 257.85 + 458.69 + 39.11) * 1e6,
-                  "source": "gemm_sm100.cu", "sha256_16": "172fbb8387d04c10"},
-    "ecdit": {"bytes": (1240.62 + 251.51 + 1483.07 + 58.34) * 1e6,
-              "source": "gemm_sm100.cu", "sha256_16": "172fbb8387d04c10"},
-    "mmoe": {"bytes": (231.53 + 154.65 + 421.11 + 40.28) * 1e6,
-             "source": "gemm_sm100.cu", "sha256_16": "172fbb8387d04c10"},
+    "ditmoe_xl": {"bytes": (163.05 + 256.27 + 458.77 + 38.32) * 1e6,
+                  "source": "gemm_sm100.cu", "sha256_16": "50f55cd1774947d4"},
+    "ecdit": {"bytes": (1230.38 + 252.20 + 1472.19 + 58.26) * 1e6,
+              "source": "gemm_sm100.cu", "sha256_16": "50f55cd1774947d4"},
+    "mmoe": {"bytes": (231.54 + 154.38 + 421.32 + 40.01) * 1e6,
+             "source": "gemm_sm100.cu", "sha256_16": "50f55cd1774947d4"},
 }
 
 

@@ -28,13 +28,15 @@
  *   - The library allocates no memory on a call's path. Scratch comes from
  *     a caller workspace of at least moe_workspace_size() bytes, 256-byte
  *     aligned. Calls that share a workspace must not overlap on the device.
- *     Two exceptions, each documented at its entry point: the
+ *     Three exceptions, each documented at its entry point: the
  *     allocation-free dispatch (moe_dispatch_noalloc) keeps its scratch in
  *     one fixed library-owned device array per GPU, shared by all its
- *     calls; and moe_forward_host creates two library-owned side streams
- *     and events per device on its first pipelined call and keeps them for
- *     the life of the process.
- *   - Apart from those two and from one-time lookups made safely on first
+ *     calls; moe_forward_host creates two library-owned side streams and
+ *     events per device on its first pipelined call; and moe_forward, for
+ *     a bf16 layer with a shared expert and routed rows, creates one
+ *     library-owned side stream and two events per device on first use.
+ *     Both keep them for the life of the process.
+ *   - Apart from those and from one-time lookups made safely on first
  *     use, there is no global mutable state: calls on different streams
  *     with different workspaces may run concurrently.
  *
@@ -398,8 +400,17 @@ typedef struct moe_forward_aux {
 
 /*
  * The whole layer: router -> selection -> dispatch -> grouped MLP ->
- * combine, every step a kernel of this library, all on `stream`, no host
- * synchronisation (group sizes stay on the device).
+ * combine, every step a kernel of this library, no host synchronisation
+ * (group sizes stay on the device). Everything runs on `stream`, except
+ * that a bf16 layer with a shared expert and routed rows (not a small
+ * block) runs the shared expert's up projection on a library-owned side
+ * stream. That stream forks from `stream` after the routing and joins it
+ * before the down projections, so the call is still ordered on `stream`
+ * as a whole, and stream capture takes the side stream in. The first
+ * such call on a device creates the side stream and its events; capture
+ * that first call only in a capture mode that allows stream and event
+ * creation. Concurrent callers on one device serialise on a host mutex
+ * while they enqueue the layer.
  *   x [T, d], residual [T, d] nullable, z_prev [T, E] fp32 nullable,
  *   W_r [E, d], bias [E] fp32 nullable, W1, W2, Ws1, Ws2 as in
  *   moe_grouped_mlp, const_vecs [n_const, d] nullable, y [T, d] out.
