@@ -504,6 +504,7 @@ template <int BN, int ACT, bool OUT_F32, int STAGES, int NH>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                         const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                          const ParamsDev p) {
   static_assert(NH == 1 || (NH == 2 && ACT != kActSwiglu), "two MMAs per k-step only without gating");
   constexpr int BMP = 2 * BM;                              // rows per pair tile
@@ -532,6 +533,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
                                               ~(uintptr_t)1023);
   const uint32_t sA = smem_u32(base);
   const uint32_t sB = sA + STAGES * A_BYTES;
+  const uint32_t sO = sB + STAGES * NH * B_BYTES;  // the epilogue warps' staging tiles
   const uint32_t full0 = smem_u32(&bars[0]);
   const uint32_t empty0 = smem_u32(&bars[STAGES]);
   const uint32_t tfull0 = smem_u32(&bars[2 * STAGES]);
@@ -678,6 +680,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
     const int quad = warp & 3;                  // TMEM lanes this warp may read
     const int lrow = quad * 32 + lane;
     const int c_lo = ((warp - 2) / 4) * (TNO / 2);  // this warp's half of the columns
+    const uint32_t stg = sO + (uint32_t)(warp - 2) * kStageOutBytes;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = seq.next(); t >= 0; t = seq.next()) {
@@ -689,6 +692,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
       const int row = sched.row0[e] + mt * BMP + (int)rank * BM + lrow;
       const bool valid = row < sched.row_end[e];
       const int col0 = nt * TNO;
+      // Whole 32-row blocks go out as TMA tile stores, a block reaching past
+      // the group's last row as per-lane stores of its valid rows.
+      const int wrow0 = sched.row0[e] + mt * BMP + (int)rank * BM + quad * 32;
+      const bool tma_rows = !OUT_F32 && pr.tma_out && wrow0 + 32 <= sched.row_end[e];
+      const CUtensorMap *mO = sched.prob[e] ? &tmO1 : &tmO0;
       const bool ready = mbar_wait_cluster(tfull0 + 8 * acc, acc_phase, &abort_flag, p.status);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
@@ -706,13 +714,26 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_
 #pragma unroll
           for (int i = 0; i < 32; i += 2) gelu_erf_x2(v[i], v[i + 1]);
         }
-        if (valid) store_row32<OUT_F32>(pr, row, col0 + c, v);
+        if (tma_rows) {
+          if (lane == 0) bulk_wait_read_all();  // the tile's previous store has read it
+          __syncwarp();
+          stage_row32_bf16(pr, row, col0 + c, v, stg, lane);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(mO, col0 + c, wrow0, stg);
+            bulk_commit();
+          }
+        } else if (valid) {
+          store_row32<OUT_F32>(pr, row, col0 + c, v);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + 8 * acc);
       if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait_all();  // every tile store has landed before the CTA exits
   }
 
   tc_fence_before();
@@ -834,10 +855,11 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
   constexpr int S0 = (200 * 1024) / STAGE_BYTES;
   constexpr int STAGES = S0 > 8 ? 8 : S0;
   constexpr int BNO = NH * ((ACT == kActSwiglu) ? BN / 2 : BN);  // output columns per tile
-  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES;
+  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + (OUT_F32 ? 0 : kEpiWarps * kStageOutBytes);
 
-  CUtensorMap maps[4];
+  CUtensorMap maps[4], omaps[2];
   memset(maps, 0, sizeof(maps));
+  memset(omaps, 0, sizeof(omaps));
   ParamsDev pd;
   memset(&pd, 0, sizeof(pd));
   pd.n_probs = n_probs;
@@ -859,9 +881,13 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
     pd.pr[i].vec32 = vec32_ok(q, OUT_F32 ? 4 : 2);
     pd.pr[i].residual = static_cast<const __nv_bfloat16 *>(q.residual);
     pd.pr[i].ld_res = q.ld_res;
+    // TMA-stored tiles on the narrow form only: the wide form's single
+    // accumulator keeps its epilogue on the critical path, where waiting for
+    // a staging tile to be read measured no better than per-lane stores.
+    pd.pr[i].tma_out = !OUT_F32 && NH == 1 && make_out_map(&omaps[i], q);
     max_tiles += max_m_tiles(q, 2 * BM) * ((q.N + BNO - 1) / BNO);
   }
-  if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; }
+  if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; omaps[1] = omaps[0]; }
   if (max_tiles == 0) return MOE_OK;
   auto kern = grouped_gemm_pair_kernel<BN, ACT, OUT_F32, STAGES, NH>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
@@ -890,7 +916,7 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
   if (clusters < 1) return MOE_ERR_UNSUPPORTED;
   if (max_tiles < clusters) clusters = (int)max_tiles;
   cfg.gridDim = dim3(2 * (unsigned)clusters);
-  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], pd));
+  MOE_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], omaps[0], omaps[1], pd));
   return last_launch_status();
 }
 
@@ -913,17 +939,23 @@ static int pick_bn(const GemmProblem *probs, int n_probs, int act) {
   return 128;
 }
 
-// The pair (2-SM) kernel pays off with full 256-wide tiles, long K (so the
-// pair's shared accumulator hand-off is amortised) and groups large enough
-// to fill 256-row tiles; measured on B200 it is slower with N=192 tiles or
-// K ~ 1152, where the single-SM kernel is used.
+// The pair (2-SM) kernel pays off with full 256-wide tiles and groups large
+// enough to fill 256-row tiles; measured on B200 it is slower with N=192
+// tiles. With short K (~1152) it beat the single-SM kernel on DiT-MoE-XL's
+// up projection (16384 assignments over 8 experts: layer 0.584 -> 0.571 ms)
+// but lost on MMOE's (16384 over 16 heavy experts, ~860 rows each once the
+// zero-computation experts take theirs: 0.431 -> 0.435 ms), whose 256-row
+// tiles leave twice the ragged rows of 128-row ones. So short K takes the
+// pair only when every problem has at least 1536 rows (assignments, an
+// upper bound on the host) per group on average.
 static bool use_pair(const GemmProblem *probs, int n_probs, int bn) {
   if (bn != 256) return false;
   int64_t rows = 0, groups = 0;
   for (int i = 0; i < n_probs; ++i) {
-    if (probs[i].K < 2048) return false;
+    const int64_t g = probs[i].offsets ? probs[i].n_groups : 1;
+    if (probs[i].K < 2048 && probs[i].a_rows < 1536 * g) return false;
     rows += probs[i].a_rows;
-    groups += probs[i].offsets ? probs[i].n_groups : 1;
+    groups += g;
   }
   return groups > 0 && rows >= 256 * groups;
 }
@@ -999,11 +1031,15 @@ static int pick_wide(const GemmProblem *probs, int n_probs, int act, int bn, boo
 }
 
 int launch_grouped_gemm_bf16(const GemmProblem *probs, int n_probs, int act, bool out_f32,
-                             int32_t *dev_status, cudaStream_t stream) {
+                             int32_t *dev_status, cudaStream_t stream, const GemmProblem *also) {
   if (n_probs < 1 || n_probs > 2) return MOE_ERR_INVALID_ARG;
   if (out_f32) return MOE_ERR_UNSUPPORTED;  // bf16 layers keep every GEMM output in bf16
-  const int bn = pick_bn(probs, n_probs, act);
-  const bool pair = use_pair(probs, n_probs, bn);
+  GemmProblem rule[3];
+  int n_rule = 0;
+  for (int i = 0; i < n_probs; ++i) rule[n_rule++] = probs[i];
+  if (also) rule[n_rule++] = *also;
+  const int bn = pick_bn(rule, n_rule, act);
+  const bool pair = use_pair(rule, n_rule, bn);
   const int wide = pick_wide(probs, n_probs, act, bn, pair);
   if (wide == 256) return run_tc_pair<256, kActNone, false, 2>(probs, n_probs, dev_status, stream);
   if (wide == 192) return run_tc_pair<192, kActNone, false, 2>(probs, n_probs, dev_status, stream);

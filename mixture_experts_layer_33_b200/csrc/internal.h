@@ -215,9 +215,13 @@ struct GemmProblem {
 inline int64_t max_m_tiles(const GemmProblem &p, int bm) {
   return (p.a_rows + bm - 1) / bm + (p.offsets ? p.n_groups : 0);
 }
+// `also` (nullable): a problem of the same activation that would share this
+// launch but runs in another one (moe_forward's shared up projection on its
+// side stream, beside the routed one); the tile shape is chosen over both,
+// so the two launches run the same kernel.
 int launch_grouped_gemm_bf16(const GemmProblem *probs, int n_probs, int act,
                              bool out_f32, int32_t *dev_status,
-                             cudaStream_t stream);
+                             cudaStream_t stream, const GemmProblem *also = nullptr);
 
 // 2-D bf16 TMA descriptor [rows, cols] (cols contiguous), box {64, box_rows},
 // 128-byte swizzle, zero fill outside the tensor.

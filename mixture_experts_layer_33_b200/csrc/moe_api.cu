@@ -329,6 +329,18 @@ GemmProblem shared_up_problem(const moe_config &c, const void *x, const void *Ws
   return g;
 }
 
+// The routed experts' up projection: H = act(x_perm W1_g^T) per group.
+GemmProblem routed_up_problem(const moe_config &c, const void *x_perm, const int32_t *offsets,
+                              const void *W1, void *H, int32_t *dev_status) {
+  const bool gated = c.act == MOE_SWIGLU;
+  GemmProblem g{};
+  g.A = x_perm; g.a_rows = n_assign_of(c); g.B = W1; g.n_groups = c.n_heavy; g.offsets = offsets;
+  g.N = c.h; g.b_rows_per_group = gated ? 2 * c.h : c.h; g.K = c.d;
+  g.out = H; g.ld_out = c.h;
+  g.status = dev_status;
+  return g;
+}
+
 // `side`: the shared up projection already runs on a forked side stream;
 // the routed up projection runs alone and the down projections wait for
 // the side stream.
@@ -345,9 +357,7 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
   const int act1 = c.act == MOE_SWIGLU ? kActSwiglu : kActGelu;
 
   GemmProblem g1r{}, g1s{}, g2r{}, g2s{};
-  g1r.A = x_perm; g1r.a_rows = na; g1r.B = W1; g1r.n_groups = c.n_heavy; g1r.offsets = offsets;
-  g1r.N = c.h; g1r.b_rows_per_group = act1 == kActSwiglu ? 2 * c.h : c.h; g1r.K = c.d;
-  g1r.out = H; g1r.ld_out = c.h;
+  g1r = routed_up_problem(c, x_perm, offsets, W1, H, dev_status);
   g2r.A = H; g2r.a_rows = na; g2r.B = W2; g2r.n_groups = c.n_heavy; g2r.offsets = offsets;
   g2r.N = c.d; g2r.b_rows_per_group = c.d; g2r.K = c.h; g2r.out = y_perm; g2r.ld_out = c.d;
   g1s = shared_up_problem(c, x, Ws1, H_sh, dev_status);
@@ -373,7 +383,9 @@ int run_grouped_mlp(const moe_config &c, const void *x_perm, const int32_t *offs
   if (c.dtype == MOE_BF16) {
     // GEMM1 (+activation): routed and shared in one tile stream when they share the activation.
     if (side) {
-      if (routed) st = launch_grouped_gemm_bf16(&g1r, 1, act1, false, dev_status, stream);
+      if (routed)
+        st = launch_grouped_gemm_bf16(&g1r, 1, act1, false, dev_status, stream,
+                                      act1 == kActGelu ? &g1s : nullptr);
       if (st == MOE_OK) st = side->join();
     } else if (routed && shared && act1 == kActGelu) {
       GemmProblem p1[2] = {g1r, g1s};
@@ -593,7 +605,9 @@ int forward_device(const moe_config &c, const void *x, const void *residual,
     st = side.fork();
     if (st != MOE_OK) return st;
     const GemmProblem g1s = shared_up_problem(c, x, Ws1, at<void>(ws, L.H_sh), dev_status);
-    st = launch_grouped_gemm_bf16(&g1s, 1, kActGelu, false, dev_status, side.side());
+    const GemmProblem g1r = routed_up_problem(c, x_perm, offsets, W1, at<void>(ws, L.H), dev_status);
+    st = launch_grouped_gemm_bf16(&g1s, 1, kActGelu, false, dev_status, side.side(),
+                                  c.act == MOE_SWIGLU ? nullptr : &g1r);
     if (st != MOE_OK) return st;
   }
   stage.next("moe_forward/dispatch");
