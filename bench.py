@@ -107,7 +107,11 @@ def forward_launches(cfg):
     r = cfg["routing"]
     ec = r == "expert_choice"
     na = (cfg["T"] // cfg["group_size"]) * cfg["E"] * cfg["capacity"] if ec else cfg["T"] * cfg["k"]
-    n = 1 + StagedLayer._mlp_launches(cfg)  # combine + expert MLP
+    if bf16 and cfg["T"] > 128 and cfg["n_shared"] and cfg["E_heavy"]:
+        # shared up projection (side stream), routed up projection, both down projections
+        n = 1 + 3
+    else:
+        n = 1 + StagedLayer._mlp_launches(cfg)  # combine + expert MLP
     if (bf16 and cfg["T"] <= 128 and r in ("token_topk", "des_vote") and cfg["E"] <= 128
             and cfg["k"] <= 32 and cfg["T"] * cfg["k"] <= 2048):
         return n + 2  # split router, then routing + dispatch + gather in one kernel
@@ -115,7 +119,10 @@ def forward_launches(cfg):
         n += 2 + (r == "des_vote")  # split router, finish (+ DES re-route)
     else:
         n += 1 + (r != "token_topk")  # router (+ expert choice / DES vote)
-    n += (1 if na <= 1024 else 3) + (1 if ec else 0)  # dispatch (+ token lists)
+    if ec and (2 * cfg["group_size"] + cfg["E"] * cfg["capacity"]) * 4 <= 48 * 1024:
+        n += 1  # closed-form expert-choice dispatch with its token lists, one launch
+    else:
+        n += (1 if na <= 1024 else 3) + (1 if ec else 0)  # dispatch (+ token lists)
     n += 1 if cfg["E_heavy"] else 0  # row gather
     return n
 
