@@ -403,6 +403,11 @@ EDGE = [
     # K = 4096 before routed K = 2048, ragged groups) and 256 x 512 tiles
     # (N = 1024, expert choice)
     ("gemm2_pair_two_mma_384", "ditmoe_xl", dict(T=3000, d=768, h=2048, h_shared=2048)),
+    # up projections with short K (256) on CTA pairs, since every problem
+    # averages >= 1536 rows per group: 256 x 256 tiles stored by TMA, the
+    # 32-row blocks past each expert's ragged end stored per lane, and the
+    # shared expert's launch (side stream) on the same kernel
+    ("gemm1_pair_short_k", "ditmoe_xl", dict(T=4100, d=256, E=4, k=2, h=512, h_shared=256)),
     ("gemm2_pair_two_mma_512", "ecdit", dict(T=16 * 128, group_size=128, d=1024, E=8, h=2048, capacity=32)),
     # 160 wide (256 x 512) down-projection tiles over 74 CTA pairs: a last
     # wave of 12 tiles on a grid of many pairs
