@@ -34,13 +34,15 @@ constexpr int kBK = 64;        // model-width slice per pipeline stage
 constexpr int kLDS = kBK + 8;  // padded smem row (bf16): conflict-free ldmatrix
 constexpr int kThreads = 128;
 constexpr int kRowwiseMaxTokens = 512;  // bf16 layers this small use one CTA per token
-constexpr int kMmaBM = 32;               // tokens per CTA of the MMA router (2 warps x 16)
-constexpr int kMmaThreads = 64;
-// cp.async ring depth: with up to 32 experts twelve 64-wide slices of the
-// token tile are in flight per CTA (a 1152-wide tile in 1.5 round trips);
-// wider expert tiles keep six to stay within shared memory.
+constexpr int kMmaBM = 32;               // tokens per CTA of the MMA router (two halves of 16)
+constexpr int kMmaWarps = 4;             // two 16-token halves x two K parities
+constexpr int kMmaThreads = 32 * kMmaWarps;
+// cp.async ring depth: up to 16 experts, twelve 64-wide slices of the
+// token tile in flight per CTA (a 1152-wide tile in 1.5 round trips);
+// 17-32 experts, eleven, so that two CTAs still fit on an SM; wider expert
+// tiles keep six to stay within shared memory.
 template <int NT>
-constexpr int mma_stages() { return NT <= 4 ? 12 : 6; }
+constexpr int mma_stages() { return NT <= 2 ? 12 : NT <= 4 ? 11 : 6; }
 
 // Softmax of one token row held by a warp: expert e = lane + 32*v.
 template <int VPL>
@@ -111,7 +113,7 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
   extern __shared__ __align__(16) unsigned char smem_raw[];
   __nv_bfloat16 *sX = reinterpret_cast<__nv_bfloat16 *>(smem_raw);   // [stages][kMmaBM][kLDS]
   __nv_bfloat16 *sW = sX + kMmaStages * kMmaBM * kLDS;                      // [stages][EP][kLDS]
-  float *sZ = reinterpret_cast<float *>(sW + kMmaStages * EP * kLDS);    // [kMmaBM][EP + 1]
+  float *sZ = reinterpret_cast<float *>(sW + kMmaStages * EP * kLDS);    // [2][kMmaBM][EP + 1]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (PARTIAL && blockIdx.x == 0 && blockIdx.y == 0) {
@@ -162,10 +164,12 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
       cp_async_commit();
     }
     const int st = kb % kMmaStages;
-    const __nv_bfloat16 *tX = sX + (st * kMmaBM + warp * 16) * kLDS;
+    // Warp w takes tokens (w & 1) * 16 .. +15 and the k16 steps of parity
+    // w >> 1; the two parities' sums are added once at the end.
+    const __nv_bfloat16 *tX = sX + (st * kMmaBM + (warp & 1) * 16) * kLDS;
     const __nv_bfloat16 *tW = sW + st * EP * kLDS;
 #pragma unroll
-    for (int kk = 0; kk < kBK / 16; ++kk) {
+    for (int kk = warp >> 1; kk < kBK / 16; kk += 2) {
       uint32_t a[4];
       ldmatrix_x4(a, tX + (lane & 15) * kLDS + kk * 16 + (lane >> 4) * 8);
 #pragma unroll
@@ -178,18 +182,22 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
   }
   cp_async_wait<0>();
 
-  // Park the 64 x EP logits tile in shared memory.
+  // Park the two K parities' kMmaBM x EP sums in shared memory, then add
+  // them (even + odd, the same order for every element).
   {
-    const int r0 = warp * 16 + (lane >> 2);
+    const int r0 = (warp & 1) * 16 + (lane >> 2);
+    float *z = sZ + (warp >> 1) * kMmaBM * (EP + 1);
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       const int c0 = n * 8 + (lane & 3) * 2;
-      sZ[r0 * (EP + 1) + c0] = acc[n][0];
-      sZ[r0 * (EP + 1) + c0 + 1] = acc[n][1];
-      sZ[(r0 + 8) * (EP + 1) + c0] = acc[n][2];
-      sZ[(r0 + 8) * (EP + 1) + c0 + 1] = acc[n][3];
+      z[r0 * (EP + 1) + c0] = acc[n][0];
+      z[r0 * (EP + 1) + c0 + 1] = acc[n][1];
+      z[(r0 + 8) * (EP + 1) + c0] = acc[n][2];
+      z[(r0 + 8) * (EP + 1) + c0 + 1] = acc[n][3];
     }
   }
+  __syncthreads();
+  for (int i = tid; i < kMmaBM * (EP + 1); i += kMmaThreads) sZ[i] += sZ[kMmaBM * (EP + 1) + i];
   __syncthreads();
   if (PARTIAL) {
     float *part = logits + (size_t)blockIdx.y * T * E;
@@ -254,8 +262,8 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
       }
     }
   } else {
-    for (int i = 0; i < 16; ++i) {
-      const int r = warp * 16 + i, s = t0 + r;
+    for (int i = 0; i < kMmaBM / kMmaWarps; ++i) {
+      const int r = warp * (kMmaBM / kMmaWarps) + i, s = t0 + r;
       if (s >= T) break;
       float z[VPL], A[VPL];
 #pragma unroll
@@ -501,7 +509,7 @@ int run_router_bf16(const void *x, const void *Wr, const float *bias, const floa
   constexpr int EP = NT * 8;
   constexpr int kMmaStages = mma_stages<NT>();
   const size_t smem = (size_t)kMmaStages * (kMmaBM + EP) * kLDS * sizeof(__nv_bfloat16) +
-                      (size_t)kMmaBM * (EP + 1) * sizeof(float);
+                      2 * (size_t)kMmaBM * (EP + 1) * sizeof(float);
   auto kern = router_bf16_kernel<NT>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   dim3 grid((T + kMmaBM - 1) / kMmaBM);
@@ -517,7 +525,7 @@ int run_router_partial(const void *x, const void *Wr, int T, int d, int E, float
   constexpr int EP = NT * 8;
   constexpr int kMmaStages = mma_stages<NT>();
   const size_t smem = (size_t)kMmaStages * (kMmaBM + EP) * kLDS * sizeof(__nv_bfloat16) +
-                      (size_t)kMmaBM * (EP + 1) * sizeof(float);
+                      2 * (size_t)kMmaBM * (EP + 1) * sizeof(float);
   auto kern = router_bf16_kernel<NT, true>;
   MOE_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   dim3 grid((T + kMmaBM - 1) / kMmaBM, n_part);
