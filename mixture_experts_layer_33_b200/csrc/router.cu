@@ -209,57 +209,74 @@ router_bf16_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__r
   }
 
   if constexpr (EP <= 32) {
-    // E <= 32: one thread per token finishes softmax and top-k serially
-    // (no shuffle chains); ties go to the lower expert id.
-    const int r = tid, s = t0 + r;
-    if (r < kMmaBM && s < T) {
-      float z[EP];
-      float m = -INFINITY;
+    // E <= 32: four lanes per token (tid / 4 is the token, tid % 4 the
+    // lane in its quad), each holding experts q, q + 4, ...; the max, the
+    // sum and each top-k round reduce over the quad with two shuffles.
+    // Ties go to the lower expert id.
+    constexpr int PER = EP / 4;
+    static_assert(EP % 4 == 0 && kMmaThreads == 4 * kMmaBM, "a quad of lanes per token");
+    const int r = tid >> 2, q = tid & 3, s = t0 + r;
+    const bool live = s < T;
+    float z[PER], A[PER];
+    float m = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        float zz = -INFINITY;
-        if (e < E) {
-          zz = sZ[r * (EP + 1) + e];
+    for (int j = 0; j < PER; ++j) {
+      const int e = q + 4 * j;
+      float zz = -INFINITY;
+      if (e < E) {
+        zz = sZ[r * (EP + 1) + e];
+        if (live) {
           if (bias) zz += bias[e];
           if (zprev) zz += zscale * zprev[(size_t)s * E + e];
           logits[(size_t)s * E + e] = zz;
-          m = fmaxf(m, zz);
         }
-        z[e] = zz;
+        m = fmaxf(m, zz);
       }
-      float A[EP];
-      float sum = 0.f;
+      z[j] = zz;
+    }
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    float sum = 0.f;
 #pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        A[e] = e < E ? expf(z[e] - m) : 0.f;
-        sum += A[e];
-      }
+    for (int j = 0; j < PER; ++j) {
+      A[j] = q + 4 * j < E ? expf(z[j] - m) : 0.f;
+      sum += A[j];
+    }
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
 #pragma unroll
-      for (int e = 0; e < EP; ++e) {
-        A[e] = A[e] / sum;
-        if (e < E) probs[(size_t)s * E + e] = A[e];
-      }
-      if (k > 0) {
-        uint32_t taken = 0;
-        float wsum = 0.f;
-        for (int j = 0; j < k; ++j) {
-          float bv = -INFINITY;
-          int bi = 0x7fffffff;
+    for (int j = 0; j < PER; ++j) {
+      A[j] = A[j] / sum;
+      if (live && q + 4 * j < E) probs[(size_t)s * E + q + 4 * j] = A[j];
+    }
+    if (k > 0) {
+      uint32_t taken = 0;  // bit j: this lane's expert q + 4j is picked
+      float wsum = 0.f;
+      for (int jj = 0; jj < k; ++jj) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        float ba = 0.f;
 #pragma unroll
-          for (int e = 0; e < EP; ++e)
-            if (e < E && !((taken >> e) & 1u) && better(z[e], e, bv, bi)) { bv = z[e]; bi = e; }
-          taken |= 1u << bi;
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < EP; ++e)
-            if (e == bi) a = A[e];
-          idx[(size_t)s * k + j] = bi;
-          w[(size_t)s * k + j] = a;
-          wsum += a;
+        for (int j = 0; j < PER; ++j) {
+          const int e = q + 4 * j;
+          if (e < E && !((taken >> j) & 1u) && better(z[j], e, bv, bi)) { bv = z[j]; bi = e; ba = A[j]; }
         }
-        if (renorm)
-          for (int j = 0; j < k; ++j) w[(size_t)s * k + j] = w[(size_t)s * k + j] / wsum;
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          const float oa = __shfl_xor_sync(0xffffffffu, ba, off);
+          if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; ba = oa; }
+        }
+        if ((bi & 3) == q) taken |= 1u << (bi >> 2);
+        if (live && q == 0) {
+          idx[(size_t)s * k + jj] = bi;
+          w[(size_t)s * k + jj] = ba;
+        }
+        wsum += ba;
       }
+      if (renorm && live && q == 0)
+        for (int jj = 0; jj < k; ++jj) w[(size_t)s * k + jj] = w[(size_t)s * k + jj] / wsum;
     }
   } else {
     for (int i = 0; i < kMmaBM / kMmaWarps; ++i) {
