@@ -62,12 +62,12 @@ class L2Flush:
 NCU_TRAFFIC = {
     "des_vote": {"bytes": (421.70 + 3.91) * 1e6,
                  "source": "block_sm100.cu", "sha256_16": "88004149b8470bd2"},
-    "ditmoe_xl": {"bytes": (163.66 + 257.57 + 459.51 + 38.67) * 1e6,
-                  "source": "gemm_sm100.cu", "sha256_16": "a9369b3f9e0b67d5"},
-    "ecdit": {"bytes": (1272.82 + 250.75 + 1475.55 + 58.30) * 1e6,
-              "source": "gemm_sm100.cu", "sha256_16": "a9369b3f9e0b67d5"},
-    "mmoe": {"bytes": (231.68 + 154.48 + 421.30 + 40.00) * 1e6,
-             "source": "gemm_sm100.cu", "sha256_16": "a9369b3f9e0b67d5"},
+    "ditmoe_xl": {"bytes": (163.55 + 257.40 + 458.85 + 38.43) * 1e6,
+                  "source": "gemm_sm100.cu", "sha256_16": "1d623aacc28d64c9"},
+    "ecdit": {"bytes": (1234.66 + 251.09 + 1472.26 + 58.55) * 1e6,
+              "source": "gemm_sm100.cu", "sha256_16": "1d623aacc28d64c9"},
+    "mmoe": {"bytes": (231.54 + 154.37 + 421.29 + 40.01) * 1e6,
+             "source": "gemm_sm100.cu", "sha256_16": "1d623aacc28d64c9"},
 }
 
 

@@ -855,7 +855,9 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
   constexpr int S0 = (200 * 1024) / STAGE_BYTES;
   constexpr int STAGES = S0 > 8 ? 8 : S0;
   constexpr int BNO = NH * ((ACT == kActSwiglu) ? BN / 2 : BN);  // output columns per tile
-  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + (OUT_F32 ? 0 : kEpiWarps * kStageOutBytes);
+  // Staging tiles for the TMA-stored output: bf16, narrow form only.
+  constexpr bool kTmaOut = !OUT_F32 && NH == 1;
+  const size_t smem = 1024 + (size_t)STAGES * STAGE_BYTES + (kTmaOut ? kEpiWarps * kStageOutBytes : 0);
 
   CUtensorMap maps[4], omaps[2];
   memset(maps, 0, sizeof(maps));
@@ -884,7 +886,7 @@ int run_tc_pair(const GemmProblem *probs, int n_probs, int32_t *status, cudaStre
     // TMA-stored tiles on the narrow form only: the wide form's single
     // accumulator keeps its epilogue on the critical path, where waiting for
     // a staging tile to be read measured no better than per-lane stores.
-    pd.pr[i].tma_out = !OUT_F32 && NH == 1 && make_out_map(&omaps[i], q);
+    pd.pr[i].tma_out = kTmaOut && make_out_map(&omaps[i], q);
     max_tiles += max_m_tiles(q, 2 * BM) * ((q.N + BNO - 1) / BNO);
   }
   if (n_probs == 1) { maps[2] = maps[0]; maps[3] = maps[1]; omaps[1] = omaps[0]; }
