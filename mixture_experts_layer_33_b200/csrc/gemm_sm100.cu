@@ -16,9 +16,12 @@
 //   warp 1       MMA issuer: one thread issues tcgen05.mma (M=128, N=BN,
 //                K=16) into a double-buffered TMEM accumulator and frees
 //                ring slots / publishes accumulators with tcgen05.commit
-//   warps 2..5   epilogue: tcgen05.ld of the accumulator (one TMEM lane
-//                quadrant per warp), activation, rounding, global store;
-//                overlaps the next tile's MMAs
+//   warps 2..9   epilogue: tcgen05.ld of the accumulator (two warps per
+//                TMEM lane quadrant, each taking half the columns),
+//                activation, rounding; bf16 tiles go out as TMA stores
+//                from a 32 x 32 staging tile per warp (per-lane stores
+//                for rows past a group's end and for fp32); overlaps the
+//                next tile's MMAs
 // SwiGLU: the B tile holds BN/2 gate rows and the matching BN/2 up rows, so
 // one accumulator carries both halves and the epilogue forms
 // silu(gate) * up without another pass.
