@@ -132,20 +132,25 @@ def forward_launches(cfg):
 KERNEL_HEADERS = ("tc_ptx.cuh", "common.cuh")
 
 
+def code_text(text):
+    """C++/CUDA source with comments and whitespace removed: what a capture
+    of the compiled kernel depends on (the kernel sources hold no string
+    literal with a comment marker in it)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", "", text)
+
+
 def source_hash(name):
     """sha256 prefix of a kernel source together with the headers it shares,
-    with comments and whitespace removed (an edit of comments or layout does
-    not change what was profiled; the kernel sources hold no string literal
-    with a comment marker in it)."""
+    taken over their code_text (an edit of comments or layout does not
+    change what was profiled)."""
     import hashlib
-    import re
     h = hashlib.sha256()
     for part in (name,) + KERNEL_HEADERS:
         with open(os.path.join(ROOT, "mixture_experts_layer_33_b200", "csrc", part), "rb") as f:
-            text = f.read().decode()
-        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        text = re.sub(r"//[^\n]*", "", text)
-        h.update(re.sub(r"\s+", "", text).encode())
+            h.update(code_text(f.read().decode()).encode())
     return h.hexdigest()[:16]
 
 

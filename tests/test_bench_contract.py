@@ -54,3 +54,20 @@ def test_reference_arm_under_torchrun_prints_once():
     lines = _json_lines(r.stdout)
     assert len(lines) == 1
     _check_line(lines[0], 2)
+
+
+def test_capture_validity_ignores_comments_and_layout_only():
+    """A DRAM-traffic figure in the bench line stays valid while the code of
+    the captured kernel is unchanged (otherwise the line reports null):
+    comments and whitespace do not count, any token of code does."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    src = ("// header comment\n__global__ void k(int *p) {\n"
+           "  /* block\n comment */ p[0] = 1;  // trailing\n}\n")
+    same = "__global__ void k(int *p) {\n\n    p[0] = 1;\n}\n// another note\n"
+    assert bench.code_text(src) == bench.code_text(same)
+    assert bench.code_text(src) != bench.code_text(src.replace("p[0] = 1", "p[0] = 2"))
+    assert bench.code_text(src) != bench.code_text(src.replace("int *p", "int *q"))
+    for entry in bench.NCU_TRAFFIC.values():
+        assert len(bench.source_hash(entry["source"])) == 16
