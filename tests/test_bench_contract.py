@@ -1,4 +1,5 @@
-"""bench.py's reference arm on the host: one JSON line with the contract's keys.
+"""bench.py on the host: the reference arm's JSON line, and the hash that
+keys the DRAM-traffic figures to the kernel code they were captured from.
 
 `bench.py --impl reference` times the fp64 oracle on the host cores (no GPU
 needed), so its line can be checked here: the same metric, unit and
